@@ -1,0 +1,112 @@
+"""Seeded synthetic inputs for the attention forward pass.
+
+This module only draws random tensors. It holds none of the attention
+arithmetic, so both the CPU oracle and the CUDA path can take their inputs
+from it without sharing any of the method.
+
+Recipe (one rule for every workload):
+  * each tensor is drawn with its own ``torch.Generator`` seeded
+    ``1000*cfg + {0: Q, 1: K, 2: V, 3: offsets / outlier channels}``;
+  * values are drawn as float32 on the CPU and then cast to the workload's
+    dtype; the oracle reads the cast values exactly;
+  * ``kind="normal"``: Q, K, V i.i.d. N(0, 1);
+  * ``kind="k_offset"``: as normal, plus a per-(batch, kv-head, channel)
+    offset drawn from N(0, 3^2) and added to every token of K.  This models
+    the channel-wise outliers of K that the SageAttention article
+    ("又快又准，即插即用！清华8比特量化Attention…", section 挑战) reports
+    for video and image models;
+  * ``kind="outlier_channels"``: as normal, then in each of Q, K and V, for
+    every (batch, head), max(1, round(0.01*d)) channels drawn at random are
+    multiplied by 10 on all tokens (independent draws per tensor).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "attention_flops", "workload"]
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    causal: bool
+    dtype: str          # "bf16" | "fp16"
+    kind: str           # "normal" | "k_offset" | "outlier_channels"
+    seed_base: int      # 1000 * cfg for the named workloads
+    modes: tuple = ("bf16_exact", "int8_qk")
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def torch_dtype(self):
+        return {"bf16": torch.bfloat16, "fp16": torch.float16}[self.dtype]
+
+    def flops(self) -> float:
+        return attention_flops(self.B, self.Hq, self.N, self.d, self.causal)
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+def attention_flops(B: int, Hq: int, N: int, d: int, causal: bool) -> float:
+    """Algorithmic FLOPs of one forward pass: 4*B*Hq*N^2*d, halved when causal."""
+    f = 4.0 * B * Hq * N * N * d
+    return f / 2.0 if causal else f
+
+
+# The five seeded workloads.  Workload 1 is small enough for a full-matrix
+# float64 oracle in milliseconds; 2 is the single-GPU headline shape.
+WORKLOADS = {
+    1: Workload("mha_n128_d64_fp16", 1, 2, 2, 128, 64, False, "fp16", "normal", 1000),
+    2: Workload("mha_causal_b4_h32_n4096_d128", 4, 32, 32, 4096, 128, True, "bf16", "normal", 2000),
+    3: Workload("gqa_causal_b2_hq32_hkv8_n8192_d128_koffset", 2, 32, 8, 8192, 128, True, "bf16",
+                "k_offset", 3000),
+    4: Workload("mha_b2_h24_n16384_d64_outliers", 2, 24, 24, 16384, 64, False, "bf16",
+                "outlier_channels", 4000, ("int8_qk", "bf16_exact")),
+    5: Workload("gqa_causal_b1_hq32_hkv8_n131072_d128_koffset", 1, 32, 8, 131072, 128, True, "bf16",
+                "k_offset", 5000),
+}
+
+
+def workload(cfg: int) -> Workload:
+    return WORKLOADS[cfg]
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def make_inputs(w: Workload):
+    """Return (q, k, v) as CPU tensors of ``w.dtype`` in [B, H, N, d] layout."""
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    f32 = torch.float32
+    q = torch.randn((B, Hq, N, d), generator=_gen(w.seed_base + 0), dtype=f32)
+    k = torch.randn((B, Hkv, N, d), generator=_gen(w.seed_base + 1), dtype=f32)
+    v = torch.randn((B, Hkv, N, d), generator=_gen(w.seed_base + 2), dtype=f32)
+    if w.kind == "k_offset":
+        off = torch.randn((B, Hkv, 1, d), generator=_gen(w.seed_base + 3), dtype=f32) * 3.0
+        k.add_(off)
+    elif w.kind == "outlier_channels":
+        g = _gen(w.seed_base + 3)
+        n_out = max(1, round(0.01 * d))
+        for t in (q, k, v):
+            for b in range(B):
+                for h in range(t.shape[1]):
+                    ch = torch.randperm(d, generator=g)[:n_out]
+                    t[b, h][:, ch] *= 10.0
+    elif w.kind != "normal":
+        raise ValueError(f"unknown input kind {w.kind!r}")
+    dt = w.torch_dtype
+    return q.to(dt), k.to(dt), v.to(dt)
