@@ -1,0 +1,181 @@
+/*
+ * tiled_attention.h - C ABI of the B200 (sm_100a) tiled attention forward pass.
+ *
+ * The operation (all entry points below compute parts of it):
+ *
+ *   O = softmax(scale * Q K^T [+ causal mask]) V,   lse_i = ln sum_j exp(s_ij)
+ *
+ *   "注意力即一切：从 MHA 到 GQA" (bojinhu.xyz), section 2.2 gives the four steps
+ *   (scores Q K^T, softmax of the scaled scores, weighted sum of V), section
+ *   2.3 the causal mask (future positions set to -inf before the softmax),
+ *   section 3.2 the independent heads and section 5.1 the grouped K/V heads
+ *   (GQA).  Section 8.2 of the same page and the "FlashAttention" glossary
+ *   page (aiunderstanding.org; deep-dive section and FAQ) give the method:
+ *   tiles of Q, K and V in on-chip memory with an online softmax (running row
+ *   maximum and row sum, partial outputs rescaled), so the N x N score matrix
+ *   never reaches HBM, and the result is the same as the plain definition.
+ *
+ *   ATTN_MODE_INT8_QK follows the SageAttention article "又快又准，即插即用！
+ *   清华8比特量化Attention，两倍加速于FlashAttention2，各端到端任务均不掉点！",
+ *   section 技术方案: K is smoothed by subtracting its per-channel mean over
+ *   tokens, Q and K are quantised to INT8 with one scale per 128-token block,
+ *   Q K^T runs on INT8 tensor cores with int32 accumulation and is dequantised,
+ *   and P V stays in 16-bit floating point.
+ *
+ * Conventions shared by every entry point
+ *   - Layout: dense row-major [B, H, N, d] (d fastest), H = Hq for Q and O,
+ *     H = Hkv for K and V.  Query head h reads kv head h / (Hq / Hkv).
+ *   - d must be 64 or 128.  N >= 1; N need not be a multiple of 128.
+ *   - Every device pointer must be 16-byte aligned (TMA requirement).
+ *   - All buffers belong to the caller.  The library allocates no memory and
+ *     keeps no state beyond one device status word per GPU.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronise, except attn_check_status and
+ *     attn_fwd_host, which say so.
+ *   - Inputs are never modified.
+ *   - Return value: ATTN_OK (0) or a negative ATTN_ERR_* code.  Argument
+ *     errors are detected on the host before anything is launched.
+ *   - Device-side waits are bounded.  A wait that runs out sets the device
+ *     status word; the kernel returns early and its outputs are undefined.
+ *     attn_check_status() reports it as ATTN_ERR_TIMEOUT.
+ */
+#ifndef TILED_ATTENTION_H
+#define TILED_ATTENTION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_ARG = -1,          /* null pointer, N < 1, Hq % Hkv != 0, bad scale/mode/dtype */
+  ATTN_ERR_UNSUPPORTED = -2,  /* d not in {64, 128}, or sizes beyond 32-bit tensor indexing */
+  ATTN_ERR_ALIGN = -3,        /* a device pointer is not 16-byte aligned */
+  ATTN_ERR_WORKSPACE = -4,    /* workspace / scratch missing or smaller than required */
+  ATTN_ERR_LAUNCH = -5,       /* a CUDA call or kernel launch failed (see attn_last_cuda_error) */
+  ATTN_ERR_TIMEOUT = -6       /* a device-side wait ran out (reported by attn_check_status) */
+};
+
+enum attn_mode { ATTN_MODE_BF16_EXACT = 0, ATTN_MODE_INT8_QK = 1 };
+enum attn_dtype { ATTN_BF16 = 0, ATTN_FP16 = 1 };
+
+/*
+ * attn_fwd - the whole forward pass.
+ *
+ *   q [B,Hq,N,d], k [B,Hkv,N,d], v [B,Hkv,N,d]: device, dtype `dtype`.
+ *   o [B,Hq,N,d]: device, written, dtype `dtype`.
+ *   lse [B,Hq,N]: device float32, written; NULL skips it.  In INT8 mode lse
+ *     includes the term scale*q_i.mean(K) that smoothing removes, so it is
+ *     the log-sum-exp of the caller's scores in both modes.
+ *   causal: 0 or 1 (key j is visible to query i when j <= i).
+ *   scale: the softmax scale (finite, > 0), normally 1/sqrt(d).
+ *   mode: ATTN_MODE_BF16_EXACT (16-bit Q K^T on tensor cores, fp32
+ *     accumulation) or ATTN_MODE_INT8_QK (runs the pre-pass of
+ *     attn_quant_smooth_k into `workspace`, then INT8 Q K^T).
+ *   workspace / ws_bytes: device memory of at least
+ *     attn_workspace_bytes(B,Hq,Hkv,N,d,mode) bytes (0 for BF16_EXACT, where
+ *     workspace may be NULL).  Its content on entry does not matter.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int N, int d, int causal, float scale, int mode,
+             int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace attn_fwd needs for these sizes and mode (0 for BF16_EXACT). */
+size_t attn_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int mode);
+
+/*
+ * attn_quant_smooth_k - the INT8 pre-pass alone (SageAttention article,
+ * section 技术方案, items on K smoothing and per-block INT8 quantisation).
+ *
+ *   kmean [B,Hkv,d] float32: per channel mean of K over all N tokens.  Sum
+ *     order (reproducible bit for bit): within each 128-token block the tokens
+ *     are added in ascending order into a float64 partial; the partials are
+ *     added in ascending block order into a float64 total; the mean is
+ *     (float)(total / N).
+ *   k8 [B,Hkv,N,d] int8, sk [B,Hkv,ceil(N/128)] float32: ks = (float)k - kmean;
+ *     per 128-token block (all d channels) amax = max|ks|, sk = amax/127,
+ *     k8 = clamp(rint(ks * (127/amax)), -127, 127), ties to even; an all-zero
+ *     block gives sk = 0 and k8 = 0.
+ *   q8 [B,Hq,N,d] int8, sq [B,Hq,ceil(N/128)] float32: the same per-block
+ *     quantisation applied to Q without smoothing.
+ *   lse_bias [B,Hq,N] float32: scale * sum_c q[i,c] * kmean[g(h),c].
+ *   scratch / scratch_bytes: device memory of at least
+ *     attn_quant_scratch_bytes(B,Hkv,N,d) bytes (float64 block partials).
+ *   q8, sq, k8, sk, kmean and lse_bias are device buffers written by the call.
+ */
+int attn_quant_smooth_k(const void* q, const void* k, int B, int Hq, int Hkv, int N, int d,
+                        int dtype, float scale, int8_t* q8, float* sq, int8_t* k8, float* sk,
+                        float* kmean, float* lse_bias, void* scratch, size_t scratch_bytes,
+                        void* stream);
+
+/* Bytes of scratch attn_quant_smooth_k needs: B*Hkv*ceil(N/128)*d*8 (+ alignment). */
+size_t attn_quant_scratch_bytes(int B, int Hkv, int N, int d);
+
+/*
+ * attn_fwd_int8_quantized - the fused INT8 attention kernel alone, on the
+ * outputs of attn_quant_smooth_k (q8, sq, k8, sk, lse_bias; all device).
+ * v, o and lse as in attn_fwd.  lse_bias may be NULL only when lse is NULL.
+ */
+int attn_fwd_int8_quantized(const int8_t* q8, const float* sq, const int8_t* k8,
+                            const float* sk, const float* lse_bias, const void* v, void* o,
+                            float* lse, int B, int Hq, int Hkv, int N, int d, int causal,
+                            float scale, int dtype, void* stream);
+
+/*
+ * attn_probe_qk_int32 - test hook: the exact int32 scores S = q8 k8^T of
+ * selected 128x128 tiles, computed by the same TMA staging and INT8 tcgen05
+ * MMA code the fused kernel uses, written to `out` instead of being
+ * dequantised.
+ *   tiles: device int32 array of 4*ntiles entries (b, h, m_tile, n_tile); the
+ *     tile covers query rows [128*m_tile, +128) and keys [128*n_tile, +128)
+ *     of query head h (kv head h / (Hq/Hkv)).  Each index is checked on the
+ *     device; an out-of-range tile writes zeros.
+ *   out: device int32 [ntiles, 128, 128]; rows/columns past N hold the
+ *     scores of zero-filled rows (0).
+ */
+int attn_probe_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int Hkv, int N,
+                        int d, const int32_t* tiles, int ntiles, int32_t* out, void* stream);
+
+/*
+ * attn_fwd_host - attn_fwd with HOST buffers: copies q, k, v from host memory
+ * (pinned memory makes the copies asynchronous) into the caller's device
+ * buffers dq, dk, dv, runs attn_fwd into do_ / dlse, and copies o (and lse
+ * when both lse pointers are non-NULL) back to host memory, all on `stream`.
+ * It then synchronises `stream` and returns; the host outputs are ready.
+ * One cudaMemcpyAsync per buffer.
+ */
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                  void* dq, void* dk, void* dv, void* do_, float* dlse,
+                  int B, int Hq, int Hkv, int N, int d, int causal, float scale, int mode,
+                  int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * attn_check_status - synchronises the current device, returns ATTN_OK or
+ * ATTN_ERR_TIMEOUT if a device-side wait ran out since the last call, and
+ * clears the status word.
+ */
+int attn_check_status(void);
+
+/*
+ * attn_test_wait_timeout - test hook for failure detection.  Launches one tiny kernel whose single
+ * thread waits on an mbarrier that nothing ever completes, with a limit of `limit_us`
+ * microseconds (1..1000000).  The wait gives up, sets the device status word and the kernel
+ * returns normally, so the next attn_check_status() returns ATTN_ERR_TIMEOUT and the context
+ * stays usable.  No fault, trap or hang is involved.
+ */
+int attn_test_wait_timeout(int limit_us, void* stream);
+
+/* Static, human-readable text for an ATTN_* code. */
+const char* attn_error_string(int code);
+
+/* The last CUDA error text seen by the library on this thread ("" if none). */
+const char* attn_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TILED_ATTENTION_H */

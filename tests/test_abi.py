@@ -1,0 +1,119 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any launch.
+No kernel runs here (there is no GPU); every call below returns during
+argument validation."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tiled_attention.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_attention_22_b200 import build, binding
+
+    build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(attn_[a-z0-9_]+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("attn_fwd", "attn_quant_smooth_k", "attn_workspace_bytes", "attn_error_string",
+                 "attn_probe_qk_int32", "attn_check_status", "attn_fwd_host", "attn_fwd_int8_quantized"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from tiled_attention_22_b200 import binding
+
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in the header but not exported"
+    assert set(declared_functions()) == set(binding.exported_symbols())
+
+
+def test_error_strings(lib):
+    for code in range(0, -7, -1):
+        assert lib.attn_error_string(code)
+    assert b"unknown" in lib.attn_error_string(-99)
+
+
+def test_workspace_sizes(lib):
+    # bf16_exact needs none; int8 holds q8, k8 (1 byte/elt), scales, mean, bias and float64 partials
+    assert lib.attn_workspace_bytes(4, 32, 32, 4096, 128, 0) == 0
+    B, Hq, Hkv, N, d = 2, 32, 8, 8192, 128
+    T = N // 128
+    need = B * Hq * N * d + B * Hkv * N * d + 4 * (B * Hq * T + B * Hkv * T + B * Hkv * d + B * Hq * N) \
+        + 8 * B * Hkv * T * d
+    got = lib.attn_workspace_bytes(B, Hq, Hkv, N, d, 1)
+    assert need <= got <= need + 7 * 256
+    assert lib.attn_quant_scratch_bytes(1, 8, 131072, 128) == 8 * 1024 * 128 * 8
+    assert lib.attn_workspace_bytes(1, 3, 2, 128, 128, 1) == 0  # Hq % Hkv != 0
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null value; never dereferenced (validation fails first)
+
+
+def _fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=2, Hkv=2, N=128, d=64, causal=0, scale=0.125,
+         mode=0, dtype=0, ws=None, ws_bytes=0):
+    return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, mode, dtype, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), -1), (dict(o=None), -1), (dict(N=0), -1), (dict(B=0), -1), (dict(Hq=3, Hkv=2), -1),
+    (dict(scale=float("nan")), -1), (dict(scale=float("inf")), -1), (dict(scale=-1.0), -1), (dict(mode=7), -1),
+    (dict(dtype=5), -1), (dict(causal=2), -1), (dict(d=96), -2), (dict(d=256), -2),
+    (dict(q=FAKE + 8), -3), (dict(v=FAKE + 2), -3), (dict(lse=FAKE + 4), -3),
+    (dict(mode=1, ws=None), -4), (dict(mode=1, ws=FAKE, ws_bytes=16), -4),
+])
+def test_attn_fwd_rejects_bad_arguments(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+
+
+def test_quant_and_probe_reject_bad_arguments(lib):
+    f = lib.attn_quant_smooth_k
+    args = [FAKE, FAKE, 1, 2, 2, 128, 64, 0, 0.125, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None]
+    bad = list(args); bad[0] = None
+    assert f(*bad) == -1
+    bad = list(args); bad[6] = 80
+    assert f(*bad) == -2
+    bad = list(args); bad[9] = FAKE + 1
+    assert f(*bad) == -3
+    bad = list(args); bad[16] = 8
+    assert f(*bad) == -4
+    p = lib.attn_probe_qk_int32
+    assert p(FAKE, FAKE, 1, 2, 2, 128, 64, FAKE, 0, FAKE, None) == -1
+    assert p(FAKE, FAKE, 1, 2, 2, 128, 48, FAKE, 1, FAKE, None) == -2
+    assert lib.attn_test_wait_timeout(0, None) == -1
+    assert lib.attn_fwd_int8_quantized(FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 2, 2, 128, 64, 0, 0.1, 0,
+                                       None) == -1
+
+
+def test_product_path_fails_loudly_without_library(tmp_path):
+    from tiled_attention_22_b200 import binding
+
+    saved = binding._lib
+    try:
+        binding._lib = None
+        with pytest.raises(RuntimeError, match="not built"):
+            binding.load_library(str(tmp_path / "missing.so"))
+    finally:
+        binding._lib = saved
+
+
+def test_product_package_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "tiled_attention_22_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn), encoding="utf-8").read()
+                assert not re.search(r"^\s*(from|import)\s+oracle", text, flags=re.M), fn

@@ -1,0 +1,296 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Tolerances (element-wise, against float64 on the same bf16/fp16 input bytes):
+  bf16_exact: max |O - O_ref| <= 2e-2, mean |O - O_ref| <= 2e-3, max |lse - lse_ref| <= 1e-3
+  int8_qk:    cosine(O, O_ref) >= 0.999 and max |O - O_ref| <= 5e-2 against exact attention,
+              the bf16_exact bounds against the INT8 emulation (same quantised scores),
+              max |lse - lse_ref| <= 5e-2
+  pre-pass:   q8, k8, sq, sk, kmean bit-exact; lse_bias within 1e-4 (+1e-4 relative)
+  int32 Q K^T: bit-exact.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attn_workloads import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+BF16_MAX, BF16_MEAN, BF16_LSE = 2e-2, 2e-3, 1e-3
+INT8_COS, INT8_MAX, INT8_LSE = 0.999, 5e-2, 5e-2
+
+
+@pytest.fixture(scope="module")
+def ta():
+    from tiled_attention_22_b200 import build
+
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import tiled_attention_22_b200 as ta
+
+    ta.attn_check_status()
+    return ta
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def gpu_fwd(ta, q, k, v, causal, mode):
+    o, l = ta.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, mode=mode)
+    torch.cuda.synchronize()
+    assert ta.attn_check_status() == 0
+    return _np(o), l.cpu().numpy().astype(np.float64)
+
+
+def assert_bf16(o, l, O, L, what=""):
+    err = np.abs(o - O)
+    assert np.isfinite(o).all(), what
+    assert err.max() <= BF16_MAX, f"{what}: max abs err {err.max():.3e}"
+    assert err.mean() <= BF16_MEAN, f"{what}: mean abs err {err.mean():.3e}"
+    assert np.abs(l - L).max() <= BF16_LSE, f"{what}: lse err {np.abs(l - L).max():.3e}"
+
+
+def cosine(a, b):
+    a, b = a.reshape(-1), b.reshape(-1)
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b) + 1e-300))
+
+
+def assert_int8(o, l, O, L, what=""):
+    assert np.isfinite(o).all(), what
+    c = cosine(o, O)
+    err = np.abs(o - O).max()
+    assert c >= INT8_COS, f"{what}: cosine {c:.6f}"
+    assert err <= INT8_MAX, f"{what}: max abs err {err:.3e}"
+    assert np.abs(l - L).max() <= INT8_LSE, f"{what}: lse err {np.abs(l - L).max():.3e}"
+
+
+def emulated(q, k, v, causal, scale, rows=None):
+    q8, sq, k8, sk, mean, bias = oracle.prepass(q, k, scale)
+    return oracle.attention_int8(q8, sq, k8, sk, bias, v, scale, causal, rows=rows)
+
+
+SMALL = [
+    # B, Hq, Hkv, N, d, causal, dtype, kind
+    (1, 2, 2, 128, 64, False, "fp16", "normal"),     # the N=128 fp16 workload's shape
+    (1, 2, 2, 128, 64, True, "fp16", "normal"),
+    (1, 2, 2, 300, 64, True, "bf16", "normal"),
+    (2, 4, 2, 515, 128, False, "bf16", "k_offset"),
+    (1, 4, 1, 257, 128, True, "fp16", "normal"),     # MQA, ragged
+    (1, 2, 2, 1, 64, False, "bf16", "normal"),       # N = 1
+    (1, 2, 2, 2, 128, True, "bf16", "normal"),
+    (1, 3, 3, 129, 64, True, "bf16", "outlier_channels"),
+    (1, 2, 2, 640, 128, True, "bf16", "k_offset"),   # several 256-row blocks, no tail
+    (1, 8, 2, 383, 128, False, "fp16", "k_offset"),
+    (1, 2, 1, 1000, 64, False, "bf16", "normal"),
+]
+
+
+def _small(case, seed):
+    B, Hq, Hkv, N, d, causal, dt, kind = case
+    w = Workload("t", B, Hq, Hkv, N, d, causal, dt, kind, seed)
+    return w, make_inputs(w)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "x".join(map(str, c)))
+def test_bf16_exact_small(ta, case):
+    w, (q, k, v) = _small(case, 70000 + SMALL.index(case) * 10)
+    o, l = gpu_fwd(ta, q, k, v, w.causal, "bf16_exact")
+    O, L = oracle.attention(q, k, v, w.scale, w.causal)
+    assert_bf16(o, l, O, L, str(case))
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "x".join(map(str, c)))
+def test_int8_qk_small(ta, case):
+    w, (q, k, v) = _small(case, 80000 + SMALL.index(case) * 10)
+    o, l = gpu_fwd(ta, q, k, v, w.causal, "int8_qk")
+    O, L = oracle.attention(q, k, v, w.scale, w.causal)
+    assert_int8(o, l, O, L, str(case))
+    Oe, Le = emulated(q, k, v, w.causal, w.scale)
+    assert_bf16(o, l, Oe, Le, "vs emulation " + str(case))
+
+
+PREPASS = [
+    (1, 2, 2, 128, 64, "fp16", "normal"),
+    (2, 4, 2, 300, 128, "bf16", "k_offset"),
+    (1, 3, 1, 1, 64, "bf16", "normal"),
+    (1, 2, 2, 515, 64, "fp16", "outlier_channels"),
+    (1, 4, 2, 2048, 128, "bf16", "k_offset"),
+]
+
+
+@pytest.mark.parametrize("case", PREPASS, ids=lambda c: "x".join(map(str, c)))
+def test_prepass_bit_exact(ta, case):
+    B, Hq, Hkv, N, d, dt, kind = case
+    w = Workload("t", B, Hq, Hkv, N, d, False, dt, kind, 90000 + PREPASS.index(case) * 10)
+    q, k, _ = make_inputs(w)
+    pre = ta.attn_quant_smooth_k(q.cuda(), k.cuda(), scale=w.scale)
+    torch.cuda.synchronize()
+    q8, sq, k8, sk, mean, bias = oracle.prepass(q, k, w.scale)
+    np.testing.assert_array_equal(pre["kmean"].cpu().numpy(), mean)
+    np.testing.assert_array_equal(pre["k8"].cpu().numpy(), k8)
+    np.testing.assert_array_equal(pre["sk"].cpu().numpy(), sk)
+    np.testing.assert_array_equal(pre["q8"].cpu().numpy(), q8)
+    np.testing.assert_array_equal(pre["sq"].cpu().numpy(), sq)
+    np.testing.assert_allclose(pre["lse_bias"].cpu().numpy(), bias, rtol=1e-4, atol=1e-4)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_int32_scores_bit_exact(ta, d):
+    w = Workload("t", 2, 4, 2, 300, d, False, "bf16", "k_offset", 95000 + d)
+    q, k, _ = make_inputs(w)
+    pre = ta.attn_quant_smooth_k(q.cuda(), k.cuda())
+    tiles = [(0, 0, 0, 0), (1, 3, 2, 1), (0, 1, 1, 2), (1, 2, 2, 2), (0, 3, 0, 2), (5, 0, 0, 0)]  # last: invalid
+    out = ta.attn_probe_qk_int32(pre["q8"], pre["k8"], tiles).cpu().numpy()
+    q8, k8 = pre["q8"].cpu().numpy(), pre["k8"].cpu().numpy()
+    N = w.N
+    for i, (b, h, m, n) in enumerate(tiles):
+        want = np.zeros((128, 128), np.int64)
+        if b < w.B:
+            acc = oracle.scores_int32(q8, k8, b, h)
+            blk = acc[m * 128:(m + 1) * 128, n * 128:(n + 1) * 128]
+            want[:blk.shape[0], :blk.shape[1]] = blk
+        np.testing.assert_array_equal(out[i], want, err_msg=str((b, h, m, n)))
+
+
+def _sample_rows(N, rng, n=12):
+    rows = {0, 1, min(127, N - 1), min(128, N - 1), N - 1, N // 2}
+    rows |= set(rng.integers(0, N, n).tolist())
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+@pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk"])
+def test_full_size_sampled_rows(ta, cfg, mode):
+    """The named workloads at full size, in the launch configuration the benchmark times; the oracle
+    computes sampled rows of sampled heads (rows are independent, so this is exact for them)."""
+    w = WORKLOADS[cfg]
+    q, k, v = make_inputs(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o, l = ta.attn_fwd(qd, kd, vd, causal=w.causal, mode=mode)
+    torch.cuda.synchronize()
+    assert ta.attn_check_status() == 0
+    rng = np.random.default_rng(cfg)
+    G = w.Hq // w.Hkv
+    heads = [(0, 0), (w.B - 1, w.Hq - 1), (int(rng.integers(w.B)), int(rng.integers(w.Hq)))]
+    o_all = []
+    O_all = []
+    for b, h in heads:
+        g = h // G
+        rows = _sample_rows(w.N, rng)
+        qs, ks, vs = q[b:b + 1, h:h + 1], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1]
+        og = _np(o[b, h, rows])[None, None]
+        lg = l[b, h, rows].cpu().numpy().astype(np.float64)[None, None]
+        O, L = oracle.attention(qs, ks, vs, w.scale, w.causal, rows=rows)
+        if mode == "bf16_exact":
+            assert_bf16(og, lg, O, L, f"cfg{cfg} b{b} h{h}")
+        else:
+            Oe, Le = emulated(qs, ks, vs, w.causal, w.scale, rows=rows)
+            assert_bf16(og, lg, Oe, Le, f"cfg{cfg} b{b} h{h} vs emulation")
+            assert np.abs(lg - L).max() <= INT8_LSE
+            assert np.abs(og - O).max() <= INT8_MAX
+            o_all.append(og.reshape(-1))
+            O_all.append(O.reshape(-1))
+    if mode == "int8_qk":
+        assert cosine(np.concatenate(o_all), np.concatenate(O_all)) >= INT8_COS
+    assert torch.isfinite(o).all()
+
+
+@pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk"])
+def test_zero_inputs(ta, mode):
+    z = torch.zeros((1, 2, 300, 128), dtype=torch.bfloat16)
+    o, l = gpu_fwd(ta, z, z, z, True, mode)
+    assert (o == 0).all()
+    np.testing.assert_allclose(l[0, 0], np.log(np.arange(1, 301)), atol=1e-4)
+
+
+@pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk"])
+def test_large_scores_exercise_rescaling(ta, mode):
+    """Scores up to a few hundred: the running max grows by more than 2^8 within rows."""
+    w = Workload("t", 1, 2, 2, 700, 64, False, "bf16", "normal", 96000)
+    q, k, v = make_inputs(w)
+    q = (q.float() * 6).to(torch.bfloat16)
+    k = (k.float() * 6 + torch.linspace(0, 3, 700)[None, None, :, None]).to(torch.bfloat16)
+    o, l = gpu_fwd(ta, q, k, v, False, mode)
+    O, L = oracle.attention(q, k, v, w.scale, False)
+    if mode == "bf16_exact":
+        assert_bf16(o, l, O, L)
+    else:
+        Oe, Le = emulated(q, k, v, False, w.scale)
+        assert np.abs(o - Oe).max() <= BF16_MAX and np.abs(l - Le).max() <= INT8_LSE
+
+
+def test_deterministic_and_gqa_equals_expanded_mha(ta):
+    w = Workload("t", 1, 8, 2, 400, 128, True, "bf16", "k_offset", 97000)
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    for mode in ("bf16_exact", "int8_qk"):
+        o1, l1 = ta.attn_fwd(q, k, v, causal=True, mode=mode)
+        o2, l2 = ta.attn_fwd(q, k, v, causal=True, mode=mode)
+        o3, l3 = ta.attn_fwd(q, k.repeat_interleave(4, dim=1).contiguous(), v.repeat_interleave(4, dim=1).contiguous(),
+                             causal=True, mode=mode)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), mode
+        assert torch.equal(o1, o3) and torch.equal(l1, l3), mode
+
+
+def test_causal_outputs_ignore_future_keys(ta):
+    w = Workload("t", 1, 2, 2, 600, 64, True, "bf16", "normal", 98000)
+    q, k, v = make_inputs(w)
+    o1, l1 = gpu_fwd(ta, q, k, v, True, "bf16_exact")
+    k2, v2 = k.clone(), v.clone()
+    k2[:, :, 300:] += 4.0
+    v2[:, :, 300:] -= 2.0
+    o2, l2 = gpu_fwd(ta, q, k2, v2, True, "bf16_exact")
+    np.testing.assert_array_equal(o1[:, :, :300], o2[:, :, :300])
+    np.testing.assert_array_equal(l1[:, :, :300], l2[:, :, :300])
+    np.testing.assert_allclose(o1[:, :, 0], _np(v[:, :, 0]), atol=1e-2)  # row 0 is V[0]
+
+
+@pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk"])
+def test_canaries_around_outputs(ta, mode):
+    """Outputs placed inside guard regions: nothing outside O and lse may change."""
+    w = Workload("t", 1, 2, 2, 333, 128, True, "bf16", "normal", 99000)
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    n_o, n_l, g = q.numel(), 2 * 333, 4096
+    obuf = torch.full((n_o + 2 * g,), 7.0, device="cuda", dtype=torch.bfloat16)
+    lbuf = torch.full((n_l + 2 * g,), -3.0, device="cuda", dtype=torch.float32)
+    o = obuf[g:g + n_o].view(q.shape)
+    l = lbuf[g:g + n_l].view(1, 2, 333)
+    ta.attn_fwd(q, k, v, causal=True, mode=mode, out=o, lse=l)
+    torch.cuda.synchronize()
+    assert (obuf[:g] == 7.0).all() and (obuf[g + n_o:] == 7.0).all()
+    assert (lbuf[:g] == -3.0).all() and (lbuf[g + n_l:] == -3.0).all()
+    assert torch.isfinite(o).all() and torch.isfinite(l).all()
+
+
+def test_host_buffer_entry_point_matches_device_call(ta):
+    w = Workload("t", 1, 4, 2, 500, 128, True, "bf16", "k_offset", 99500)
+    q, k, v = make_inputs(w)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((1, 4, 500), dtype=torch.float32).pin_memory()
+    for mode in ("bf16_exact", "int8_qk"):
+        dq, dk, dv = torch.empty_like(q, device="cuda"), torch.empty_like(k, device="cuda"), torch.empty_like(v, device="cuda")
+        do = torch.empty_like(dq)
+        dl = torch.empty((1, 4, 500), device="cuda", dtype=torch.float32)
+        ws_bytes = ta.attn_workspace_bytes(1, 4, 2, 500, 128, mode)
+        ws = torch.empty(max(ws_bytes, 1), device="cuda", dtype=torch.uint8) if ws_bytes else None
+        ta.attn_fwd_host(qh, kh, vh, oh, lh, dq, dk, dv, do, dl, causal=True, mode=mode, workspace=ws)
+        o_ref, l_ref = ta.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, mode=mode)
+        torch.cuda.synchronize()
+        assert torch.equal(oh, o_ref.cpu()) and torch.equal(lh, l_ref.cpu()), mode
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(ta):
+    ta.attn_check_status()
+    ta.attn_test_wait_timeout(2000)  # 2 ms limit on a barrier nothing completes
+    assert ta.attn_check_status() == ta.ATTN_ERR_TIMEOUT
+    assert ta.attn_check_status() == 0  # cleared
+    w = Workload("t", 1, 2, 2, 200, 64, False, "bf16", "normal", 99700)
+    q, k, v = make_inputs(w)
+    o, l = gpu_fwd(ta, q, k, v, False, "bf16_exact")
+    O, L = oracle.attention(q, k, v, w.scale, False)
+    assert_bf16(o, l, O, L)

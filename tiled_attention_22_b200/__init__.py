@@ -1,0 +1,28 @@
+"""B200 (sm_100a) tiled attention forward: bf16_exact and SageAttention-style int8_qk.
+
+The computation runs in the CUDA library built from ``csrc/`` (C ABI in
+``include/tiled_attention.h``); this package only marshals arguments.
+"""
+from .binding import (  # noqa: F401
+    ATTN_ERR_ALIGN,
+    ATTN_ERR_ARG,
+    ATTN_ERR_LAUNCH,
+    ATTN_ERR_TIMEOUT,
+    ATTN_ERR_UNSUPPORTED,
+    ATTN_ERR_WORKSPACE,
+    ATTN_OK,
+    AttnError,
+    LIB_PATH,
+    attn_check_status,
+    attn_error_string,
+    attn_fwd,
+    attn_fwd_host,
+    attn_fwd_int8_quantized,
+    attn_probe_qk_int32,
+    attn_quant_scratch_bytes,
+    attn_quant_smooth_k,
+    attn_test_wait_timeout,
+    attn_workspace_bytes,
+    exported_symbols,
+    load_library,
+)

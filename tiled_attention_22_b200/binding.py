@@ -1,0 +1,213 @@
+"""ctypes binding of include/tiled_attention.h (argument marshalling only).
+
+Every function here has the name of the C entry point it calls.  torch is used
+for device memory and streams: outputs are allocated with torch, pointers and
+the current CUDA stream are passed to the library, and every step of the
+computation runs in the library's kernels.  There is no fallback: if the built
+library is missing, or no CUDA device is present, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libtiled_attention.so")
+
+ATTN_OK = 0
+ATTN_ERR_ARG = -1
+ATTN_ERR_UNSUPPORTED = -2
+ATTN_ERR_ALIGN = -3
+ATTN_ERR_WORKSPACE = -4
+ATTN_ERR_LAUNCH = -5
+ATTN_ERR_TIMEOUT = -6
+
+MODES = {"bf16_exact": 0, "int8_qk": 1}
+DTYPES = {torch.bfloat16: 0, torch.float16: 1}
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_SIGNATURES = {
+    "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _sz, _vp]),
+    "attn_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "attn_quant_smooth_k": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "attn_quant_scratch_bytes": (_sz, [_i, _i, _i, _i]),
+    "attn_fwd_int8_quantized": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
+    "attn_probe_qk_int32": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp]),
+    "attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i,
+                           _vp, _sz, _vp]),
+    "attn_check_status": (_i, []),
+    "attn_error_string": (ctypes.c_char_p, [_i]),
+    "attn_last_cuda_error": (ctypes.c_char_p, []),
+    "attn_test_wait_timeout": (_i, [_i, _vp]),
+}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        lib = load_library()
+        msg = lib.attn_error_string(code).decode()
+        extra = lib.attn_last_cuda_error().decode() if code == ATTN_ERR_LAUNCH else ""
+        super().__init__(f"{where}: {msg} ({code}){' - ' + extra if extra else ''}")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the built library (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library not built: {path} (run python -m tiled_attention_22_b200.build)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGNATURES)
+
+
+def _check(rc: int, where: str):
+    if rc != ATTN_OK:
+        raise AttnError(rc, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _shape(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    B, Hq, N, d = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[2] != N or k.shape[3] != d:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k.shape)} v {tuple(v.shape)}")
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    if q.dtype not in DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one dtype: bfloat16 or float16")
+    return B, Hq, k.shape[1], N, d
+
+
+def attn_workspace_bytes(B, Hq, Hkv, N, d, mode="int8_qk") -> int:
+    return int(load_library().attn_workspace_bytes(B, Hq, Hkv, N, d, MODES[mode]))
+
+
+def attn_quant_scratch_bytes(B, Hkv, N, d) -> int:
+    return int(load_library().attn_quant_scratch_bytes(B, Hkv, N, d))
+
+
+def attn_fwd(q, k, v, causal=False, scale=None, mode="bf16_exact", out=None, lse=True, workspace=None,
+             stream=None):
+    """O = softmax(scale Q K^T [+causal]) V on the GPU.  Returns (o, lse or None)."""
+    lib = load_library()
+    B, Hq, Hkv, N, d = _shape(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32) if lse is True else (lse or None)
+    ws_bytes = attn_workspace_bytes(B, Hq, Hkv, N, d, mode)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    rc = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, int(bool(causal)), scale,
+                      MODES[mode], DTYPES[q.dtype], _ptr(workspace),
+                      0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "attn_fwd")
+    return o, l
+
+
+def attn_quant_smooth_k(q, k, scale=None, scratch=None, stream=None, out=None):
+    """The INT8 pre-pass alone.  Returns dict(q8, sq, k8, sk, kmean, lse_bias) (``out`` if given)."""
+    lib = load_library()
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    _shape(q, k, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    T = (N + 127) // 128
+    dev = q.device
+    out = out or dict(
+        q8=torch.empty((B, Hq, N, d), device=dev, dtype=torch.int8),
+        sq=torch.empty((B, Hq, T), device=dev, dtype=torch.float32),
+        k8=torch.empty((B, Hkv, N, d), device=dev, dtype=torch.int8),
+        sk=torch.empty((B, Hkv, T), device=dev, dtype=torch.float32),
+        kmean=torch.empty((B, Hkv, d), device=dev, dtype=torch.float32),
+        lse_bias=torch.empty((B, Hq, N), device=dev, dtype=torch.float32),
+    )
+    nbytes = attn_quant_scratch_bytes(B, Hkv, N, d)
+    if scratch is None:
+        scratch = torch.empty(nbytes, device=dev, dtype=torch.uint8)
+    rc = lib.attn_quant_smooth_k(_ptr(q), _ptr(k), B, Hq, Hkv, N, d, DTYPES[q.dtype], scale, _ptr(out["q8"]),
+                                 _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]), _ptr(out["kmean"]),
+                                 _ptr(out["lse_bias"]), _ptr(scratch), scratch.numel(), _stream(stream))
+    _check(rc, "attn_quant_smooth_k")
+    return out
+
+
+def attn_fwd_int8_quantized(pre, v, causal=False, scale=None, out=None, lse=True, stream=None):
+    """The fused INT8 kernel on the outputs of attn_quant_smooth_k (``pre``)."""
+    lib = load_library()
+    q8, k8 = pre["q8"], pre["k8"]
+    B, Hq, N, d = q8.shape
+    Hkv = k8.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty((B, Hq, N, d), device=v.device, dtype=v.dtype) if out is None else out
+    l = torch.empty((B, Hq, N), device=v.device, dtype=torch.float32) if lse is True else (lse or None)
+    rc = lib.attn_fwd_int8_quantized(_ptr(q8), _ptr(pre["sq"]), _ptr(k8), _ptr(pre["sk"]), _ptr(pre["lse_bias"]),
+                                     _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, int(bool(causal)), scale,
+                                     DTYPES[v.dtype], _stream(stream))
+    _check(rc, "attn_fwd_int8_quantized")
+    return o, l
+
+
+def attn_probe_qk_int32(q8, k8, tiles, stream=None):
+    """int32 scores of 128x128 tiles; ``tiles`` is a list of (b, h, m_tile, n_tile)."""
+    lib = load_library()
+    B, Hq, N, d = q8.shape
+    Hkv = k8.shape[1]
+    t = torch.tensor(tiles, dtype=torch.int32).reshape(-1, 4).to(q8.device)
+    out = torch.empty((t.shape[0], 128, 128), device=q8.device, dtype=torch.int32)
+    rc = lib.attn_probe_qk_int32(_ptr(q8), _ptr(k8), B, Hq, Hkv, N, d, _ptr(t), t.shape[0], _ptr(out),
+                                 _stream(stream))
+    _check(rc, "attn_probe_qk_int32")
+    return out
+
+
+def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, dq, dk, dv, do_, dlse, causal=False, scale=None,
+                  mode="bf16_exact", workspace=None, stream=None):
+    """attn_fwd with host buffers: H2D of q, k, v, the forward pass, D2H of o (and lse); synchronises."""
+    lib = load_library()
+    B, Hq, N, d = q_host.shape
+    Hkv = k_host.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib.attn_fwd_host(_ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host), _ptr(lse_host), _ptr(dq),
+                           _ptr(dk), _ptr(dv), _ptr(do_), _ptr(dlse), B, Hq, Hkv, N, d, int(bool(causal)), scale,
+                           MODES[mode], DTYPES[q_host.dtype], _ptr(workspace),
+                           0 if workspace is None else workspace.numel(), _stream(stream))
+    _check(rc, "attn_fwd_host")
+
+
+def attn_check_status() -> int:
+    """Synchronise and return (and clear) the device status: 0 or ATTN_ERR_TIMEOUT."""
+    return int(load_library().attn_check_status())
+
+
+def attn_error_string(code: int) -> str:
+    return load_library().attn_error_string(code).decode()
+
+
+def attn_test_wait_timeout(limit_us: int, stream=None) -> None:
+    _check(load_library().attn_test_wait_timeout(int(limit_us), _stream(stream)), "attn_test_wait_timeout")

@@ -1,0 +1,368 @@
+// api.cu - the C ABI declared in include/tiled_attention.h: argument checks, TMA descriptors,
+// workspace layout and kernel launches.  One translation unit holds every kernel, so the device
+// status word below is a single symbol per GPU.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "tiled_attention.h"
+
+#include "attn_fwd_kernels.cuh"
+#include "prepass_kernels.cuh"
+
+namespace {
+
+using namespace tattn;
+
+thread_local char g_last_cuda_error[256] = "";
+
+int cuda_fail(cudaError_t e, const char* what) {
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+  return ATTN_ERR_LAUNCH;
+}
+#define TATTN_CUDA(call)                             \
+  do {                                               \
+    cudaError_t e_ = (call);                         \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_shape(int B, int Hq, int Hkv, int N, int d) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_ARG;
+  if (Hq % Hkv) return ATTN_ERR_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  // kernels index with 32-bit grid coordinates and TMA rows; keep every extent well inside that
+  const long long rows = (long long)B * Hq * N;
+  if (rows > (1ll << 31) - 1 || (long long)B * Hq > (1 << 30) || N > (1 << 30)) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+// ----------------------------------------- TMA descriptors ----------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [BH, N, d] view of a [B, H, N, d] tensor; box = box_x elements x 128 rows x 1 head.
+int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
+             int box_x, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
+    return ATTN_ERR_LAUNCH;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * elem_bytes, (cuuint64_t)N * d * elem_bytes};
+  cuuint32_t box[3] = {(cuuint32_t)box_x, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return ATTN_ERR_LAUNCH;
+  }
+  return ATTN_OK;
+}
+
+CUtensorMapSwizzle swizzle_for(int row_bytes) {
+  return row_bytes >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+}
+
+// ----------------------------------------- fused kernel launch ------------------------------------
+template <int D, bool INT8, bool FP16>
+int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p, cudaStream_t stream) {
+  using C = FwdCfg<D, INT8>;
+  CUtensorMap tq, tk, tv;
+  const CUtensorMapDataType qk_dt =
+      INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : (FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  const CUtensorMapDataType v_dt = FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  int rc;
+  if ((rc = make_map(&tq, q, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hq, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
+  if ((rc = make_map(&tk, k, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hkv, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
+  if ((rc = make_map(&tv, v, v_dt, 2, D, p.N, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  auto kern = attn_fwd_kernel<D, INT8, FP16>;
+  TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  const long long grid = (long long)p.n_mblocks * p.B * p.Hq;
+  kern<<<(unsigned)grid, kFwdThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  TATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
+template <bool INT8>
+int launch_fwd(const void* q, const void* k, const void* v, int d, int dtype, const FwdParams& p,
+               cudaStream_t stream) {
+  const bool fp16 = dtype == ATTN_FP16;
+  if (d == 128) return fp16 ? launch_fwd_t<128, INT8, true>(q, k, v, p, stream) : launch_fwd_t<128, INT8, false>(q, k, v, p, stream);
+  return fp16 ? launch_fwd_t<64, INT8, true>(q, k, v, p, stream) : launch_fwd_t<64, INT8, false>(q, k, v, p, stream);
+}
+
+FwdParams make_params(int B, int Hq, int Hkv, int N, int causal, float scale, void* o, float* lse) {
+  FwdParams p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.causal = causal;
+  p.n_mblocks = (N + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = o;
+  p.lse = lse;
+  return p;
+}
+
+int check_common(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int Hq,
+                 int Hkv, int N, int d, int causal, float scale, int dtype) {
+  if (!q || !k || !v || !o) return ATTN_ERR_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_ARG;
+  int rc = check_shape(B, Hq, Hkv, N, d);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return ATTN_ERR_ALIGN;
+  return ATTN_OK;
+}
+
+// ----------------------------------------- workspace layout ---------------------------------------
+struct WsLayout {
+  size_t q8, k8, sq, sk, kmean, bias, scratch, total;
+};
+
+size_t scratch_bytes(int B, int Hkv, int N, int d) {
+  const size_t T = ((size_t)N + 127) / 128;
+  return align256((size_t)B * Hkv * T * d * sizeof(double));
+}
+
+WsLayout ws_layout(int B, int Hq, int Hkv, int N, int d) {
+  const size_t T = ((size_t)N + 127) / 128;
+  WsLayout w{};
+  size_t off = 0;
+  w.q8 = off;      off += align256((size_t)B * Hq * N * d);
+  w.k8 = off;      off += align256((size_t)B * Hkv * N * d);
+  w.sq = off;      off += align256((size_t)B * Hq * T * 4);
+  w.sk = off;      off += align256((size_t)B * Hkv * T * 4);
+  w.kmean = off;   off += align256((size_t)B * Hkv * d * 4);
+  w.bias = off;    off += align256((size_t)B * Hq * N * 4);
+  w.scratch = off; off += scratch_bytes(B, Hkv, N, d);
+  w.total = off;
+  return w;
+}
+
+int launch_prepass(const void* q, const void* k, int B, int Hq, int Hkv, int N, int d, int dtype, float scale,
+                   int8_t* q8, float* sq, int8_t* k8, float* sk, float* kmean, float* bias, double* part,
+                   cudaStream_t stream) {
+  const int T = (N + 127) / 128;
+  const int BG = B * Hkv;
+  const bool fp16 = dtype == ATTN_FP16;
+  const auto* k16 = static_cast<const uint16_t*>(k);
+  const auto* q16 = static_cast<const uint16_t*>(q);
+  {
+    const long long threads = (long long)BG * T * (d / 8);
+    const unsigned blocks = (unsigned)((threads + 127) / 128);
+    if (fp16)
+      kmean_partial_kernel<true><<<blocks, 128, 0, stream>>>(k16, BG, N, d, part);
+    else
+      kmean_partial_kernel<false><<<blocks, 128, 0, stream>>>(k16, BG, N, d, part);
+    TATTN_CUDA(cudaGetLastError());
+  }
+  kmean_final_kernel<<<(BG * d + 127) / 128, 128, 0, stream>>>(part, BG, N, d, kmean);
+  TATTN_CUDA(cudaGetLastError());
+  const unsigned qblocks = (unsigned)((long long)B * Hkv * T + (long long)B * Hq * T);
+  if (d == 128) {
+    if (fp16)
+      quant_kernel<128, true><<<qblocks, 256, 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+    else
+      quant_kernel<128, false><<<qblocks, 256, 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+  } else {
+    if (fp16)
+      quant_kernel<64, true><<<qblocks, 256, 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+    else
+      quant_kernel<64, false><<<qblocks, 256, 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+  }
+  TATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
+int fwd_int8_quantized(const int8_t* q8, const float* sq, const int8_t* k8, const float* sk, const float* bias,
+                       const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal,
+                       float scale, int dtype, cudaStream_t stream) {
+  FwdParams p = make_params(B, Hq, Hkv, N, causal, scale, o, lse);
+  p.sq = sq;
+  p.sk = sk;
+  p.bias = bias;
+  return launch_fwd<true>(q8, k8, v, d, dtype, p, stream);
+}
+
+__global__ void wait_forever_probe_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the wait must give up after limit_ns and report it
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, 0x7f, limit_ns);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t attn_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int mode) {
+  if (mode != ATTN_MODE_INT8_QK) return 0;
+  if (check_shape(B, Hq, Hkv, N, d)) return 0;
+  return ws_layout(B, Hq, Hkv, N, d).total;
+}
+
+size_t attn_quant_scratch_bytes(int B, int Hkv, int N, int d) {
+  if (B < 1 || Hkv < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  return scratch_bytes(B, Hkv, N, d);
+}
+
+int attn_quant_smooth_k(const void* q, const void* k, int B, int Hq, int Hkv, int N, int d, int dtype, float scale,
+                        int8_t* q8, float* sq, int8_t* k8, float* sk, float* kmean, float* lse_bias, void* scratch,
+                        size_t scratch_bytes_given, void* stream) {
+  if (!q || !k || !q8 || !sq || !k8 || !sk || !kmean || !lse_bias) return ATTN_ERR_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_ARG;
+  int rc = check_shape(B, Hq, Hkv, N, d);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8) || !aligned16(kmean) || !aligned16(sq) ||
+      !aligned16(sk) || !aligned16(lse_bias))
+    return ATTN_ERR_ALIGN;
+  if (!scratch || scratch_bytes_given < scratch_bytes(B, Hkv, N, d)) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(scratch)) return ATTN_ERR_ALIGN;
+  return launch_prepass(q, k, B, Hq, Hkv, N, d, dtype, scale, q8, sq, k8, sk, kmean, lse_bias,
+                        static_cast<double*>(scratch), static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_int8_quantized(const int8_t* q8, const float* sq, const int8_t* k8, const float* sk,
+                            const float* lse_bias, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                            int d, int causal, float scale, int dtype, void* stream) {
+  int rc = check_common(q8, k8, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype);
+  if (rc) return rc;
+  if (!sq || !sk || (lse && !lse_bias)) return ATTN_ERR_ARG;
+  return fwd_int8_quantized(q8, sq, k8, sk, lse_bias, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
+             int causal, float scale, int mode, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_common(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mode == ATTN_MODE_BF16_EXACT) {
+    FwdParams p = make_params(B, Hq, Hkv, N, causal, scale, o, lse);
+    return launch_fwd<false>(q, k, v, d, dtype, p, st);
+  }
+  if (mode != ATTN_MODE_INT8_QK) return ATTN_ERR_ARG;
+  const WsLayout w = ws_layout(B, Hq, Hkv, N, d);
+  if (!workspace || ws_bytes < w.total) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto* q8 = reinterpret_cast<int8_t*>(ws + w.q8);
+  auto* k8 = reinterpret_cast<int8_t*>(ws + w.k8);
+  auto* sq = reinterpret_cast<float*>(ws + w.sq);
+  auto* sk = reinterpret_cast<float*>(ws + w.sk);
+  auto* kmean = reinterpret_cast<float*>(ws + w.kmean);
+  auto* bias = reinterpret_cast<float*>(ws + w.bias);
+  auto* part = reinterpret_cast<double*>(ws + w.scratch);
+  rc = launch_prepass(q, k, B, Hq, Hkv, N, d, dtype, scale, q8, sq, k8, sk, kmean, bias, part, st);
+  if (rc) return rc;
+  return fwd_int8_quantized(q8, sq, k8, sk, bias, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype, st);
+}
+
+int attn_probe_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int Hkv, int N, int d,
+                        const int32_t* tiles, int ntiles, int32_t* out, void* stream) {
+  if (!q8 || !k8 || !tiles || !out || ntiles < 1) return ATTN_ERR_ARG;
+  int rc = check_shape(B, Hq, Hkv, N, d);
+  if (rc) return rc;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(out) || !aligned16(tiles)) return ATTN_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap tq, tk;
+  const int row = d;  // int8 row bytes
+  const int box_x = row >= 128 ? 128 : 64;
+  if ((rc = make_map(&tq, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * Hq, box_x, swizzle_for(row)))) return rc;
+  if ((rc = make_map(&tk, k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, B * Hkv, box_x, swizzle_for(row)))) return rc;
+  const int smem = 2 * 128 * d + 64 + 1024;
+  if (d == 128) {
+    probe_qk_kernel<128><<<ntiles, 160, smem, st>>>(tq, tk, B, Hq, Hkv, N, tiles, out);
+  } else {
+    probe_qk_kernel<64><<<ntiles, 160, smem, st>>>(tq, tk, B, Hq, Hkv, N, tiles, out);
+  }
+  TATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, void* dq, void* dk, void* dv,
+                  void* do_, float* dlse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, int mode,
+                  int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  if (!q || !k || !v || !o) return ATTN_ERR_ARG;
+  int rc = check_common(dq, dk, dv, do_, dlse, B, Hq, Hkv, N, d, causal, scale, dtype);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t qbytes = (size_t)B * Hq * N * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
+  TATTN_CUDA(cudaMemcpyAsync(dq, q, qbytes, cudaMemcpyHostToDevice, st));
+  TATTN_CUDA(cudaMemcpyAsync(dk, k, kvbytes, cudaMemcpyHostToDevice, st));
+  TATTN_CUDA(cudaMemcpyAsync(dv, v, kvbytes, cudaMemcpyHostToDevice, st));
+  float* dl = (lse && dlse) ? dlse : nullptr;
+  rc = attn_fwd(dq, dk, dv, do_, dl, B, Hq, Hkv, N, d, causal, scale, mode, dtype, workspace, ws_bytes, stream);
+  if (rc) return rc;
+  TATTN_CUDA(cudaMemcpyAsync(o, do_, qbytes, cudaMemcpyDeviceToHost, st));
+  if (dl) TATTN_CUDA(cudaMemcpyAsync(lse, dl, (size_t)B * Hq * N * 4, cudaMemcpyDeviceToHost, st));
+  TATTN_CUDA(cudaStreamSynchronize(st));
+  return ATTN_OK;
+}
+
+int attn_check_status(void) {
+  TATTN_CUDA(cudaDeviceSynchronize());
+  int st = 0, zero = 0;
+  TATTN_CUDA(cudaMemcpyFromSymbol(&st, tattn::g_status, sizeof(int)));
+  TATTN_CUDA(cudaMemcpyToSymbol(tattn::g_status, &zero, sizeof(int)));
+  return (st & tattn::STATUS_TIMEOUT) ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+// Test hook for failure detection: one thread waits on an mbarrier that nothing ever completes,
+// with a limit of `limit_us` microseconds, so the bounded-wait path runs without faulting the GPU.
+int attn_test_wait_timeout(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return ATTN_ERR_ARG;
+  wait_forever_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((unsigned long long)limit_us * 1000ull);
+  TATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
+const char* attn_error_string(int code) {
+  switch (code) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported size (d must be 64 or 128)";
+    case ATTN_ERR_ALIGN: return "device pointer not 16-byte aligned";
+    case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case ATTN_ERR_LAUNCH: return "CUDA launch or call failed";
+    case ATTN_ERR_TIMEOUT: return "a device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* attn_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

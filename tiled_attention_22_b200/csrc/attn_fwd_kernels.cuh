@@ -1,0 +1,533 @@
+// attn_fwd_kernels.cuh - the fused attention forward kernel for sm_100a (and the int32 score probe
+// that shares its staging and MMA code).
+//
+// What it computes: O = softmax(scale * Q K^T [+ causal mask]) V and lse, per (batch, query head),
+// with query head h reading kv head h / (Hq/Hkv) ("注意力即一切：从 MHA 到 GQA", sections 2.2, 2.3,
+// 3.2, 5.1).  How: FlashAttention's tiling with an online softmax (same page, section 8.2; the
+// "FlashAttention" glossary page, deep-dive section and FAQ): Q tiles stay on chip, K/V tiles stream
+// through shared memory, a running row maximum m and row sum l rescale the partial output, and the
+// N x N scores exist only as 128 x 128 tiles in tensor memory.  In INT8 mode the Q K^T tile is an
+// INT8 x INT8 -> int32 product of the pre-pass outputs, dequantised by sq * sk (SageAttention
+// article, section 技术方案), and P V stays in 16-bit floating point.
+//
+// B200 design (not the pages'; their kernels target Ampere/Ada/Hopper):
+//   * CTA = 2 query tiles of 128 rows, 320 threads in four roles:
+//       warps 0-3  softmax for query tile 0 (thread = one row; TMEM lanes 0..127)
+//       warps 4-7  softmax for query tile 1
+//       warp  8    TMA producer: Q tiles once, then K and V tiles through separate mbarrier rings
+//       warp  9    MMA issuer (one thread): tcgen05.mma S = Q K^T into TMEM, O += P V from TMEM
+//   * TMEM (512 columns): S/P of tile t at column 128 t; O of tile t at column 256 + t D.
+//     P (16-bit) is written over the first 64 columns of S and consumed as the A operand of P V
+//     straight from TMEM, so P never touches shared memory.
+//   * The two tiles ping-pong: while one softmax group works on its S, the tensor core runs the
+//     other tile's P V and next Q K^T.
+//   * Lazy rescaling: the running max used for exp2 moves only when a row's max grows by more than
+//     2^8; otherwise the stale max keeps p <= 256 (exact: the same m is used for l and O).
+//   * Every wait is bounded (ptx.cuh); a timeout raises a CTA abort flag, each role drains what it
+//     has in flight and TMEM is always released.
+#pragma once
+#include <climits>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace tattn {
+
+struct FwdParams {
+  int B, Hq, Hkv, N, causal;
+  int n_mblocks;          // ceil(N / 256)
+  float scale_log2;       // scale * log2(e)
+  void* o;                // [B, Hq, N, D] 16-bit
+  float* lse;             // [B, Hq, N] or null
+  const float* sq;        // INT8: [B, Hq, ceil(N/128)]
+  const float* sk;        // INT8: [B, Hkv, ceil(N/128)]
+  const float* bias;      // INT8: [B, Hq, N] (null allowed when lse is null)
+};
+
+template <int D, bool INT8>
+struct FwdCfg {
+  static constexpr int BM = 128, BN = 128, QT = 2;
+  static constexpr int QK_ELEM = INT8 ? 1 : 2;                 // bytes per Q/K element
+  static constexpr int QK_ROW = D * QK_ELEM;                   // bytes per Q/K row
+  static constexpr int QK_SPAN = QK_ROW >= 128 ? 128 : 64;     // swizzle span (bytes)
+  static constexpr uint32_t QK_SWZ = QK_SPAN == 128 ? kSwizzle128B : kSwizzle64B;
+  static constexpr int QK_PANELS = QK_ROW / QK_SPAN;           // TMA boxes per tile
+  static constexpr int QK_PANEL_BYTES = 128 * QK_SPAN;
+  static constexpr int QK_BOX_X = QK_SPAN / QK_ELEM;           // elements per box row
+  static constexpr int QK_STEPS = QK_ROW / 32;                 // 32 bytes of K per MMA
+  static constexpr int Q_TILE = BM * QK_ROW;
+  static constexpr int K_TILE = BN * QK_ROW;
+  static constexpr int V_PANELS = D / 64;                      // 64 x 16-bit = 128 B per box row
+  static constexpr int V_PANEL_BYTES = BN * 128;
+  static constexpr int V_TILE = BN * D * 2;
+  static constexpr int PV_STEPS = BN / 16;
+  static constexpr int KSTAGES = (D == 128 && !INT8) ? 2 : 4;
+  static constexpr int VSTAGES = (D == 128) ? (INT8 ? 3 : 2) : 4;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + QT * Q_TILE;
+  static constexpr int OFF_V = OFF_K + KSTAGES * K_TILE;
+  static constexpr int OFF_BAR = OFF_V + VSTAGES * V_TILE;
+  // barriers: q_full[2] k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2] o_done[2] drain
+  static constexpr int NBAR = 2 + 2 * KSTAGES + 2 * VSTAGES + 6 + 1;
+  static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
+  // +1024 for manual alignment of the dynamic shared memory base; at least 120 KB so that exactly
+  // one CTA (which owns all 512 TMEM columns) is resident per SM.
+  static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 120 * 1024 ? (SMEM_USED + 1024) : 120 * 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  __host__ __device__ static constexpr uint32_t tm_s(int t) { return 128u * t; }
+  __host__ __device__ static constexpr uint32_t tm_o(int t) { return 256u + (uint32_t)(D * t); }
+  static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
+};
+
+constexpr int kFwdThreads = 320;
+
+// Wait-site ids recorded with a timeout (role * 16 + barrier kind).
+enum : int { W_LOAD = 0x10, W_MMA = 0x20, W_SOFTMAX = 0x30, W_DRAIN = 0x40, W_PROBE = 0x50 };
+
+// Issue the QK_STEPS MMAs of S(tmem) = Q_tile * K_tile^T; both operands K-major, swizzled.
+template <int D, bool INT8, bool FP16>
+__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem) {
+  using C = FwdCfg<D, INT8>;
+  constexpr uint32_t idesc = INT8 ? instr_desc(2, 1, 0, 0, 128, 128) : instr_desc(1, FP16 ? 0 : 1, 0, 0, 128, 128);
+#pragma unroll
+  for (int kk = 0; kk < C::QK_STEPS; ++kk) {
+    const uint32_t off = (uint32_t)((kk * 32) / C::QK_SPAN) * C::QK_PANEL_BYTES + (uint32_t)((kk * 32) % C::QK_SPAN);
+    const uint64_t ad = smem_desc(q_smem + off, 16, 8 * C::QK_SPAN, C::QK_SWZ);
+    const uint64_t bd = smem_desc(k_smem + off, 16, 8 * C::QK_SPAN, C::QK_SWZ);
+    if constexpr (INT8)
+      mma_i8_ss(s_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+    else
+      mma_f16_ss(s_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// Issue O(tmem) (+)= P(tmem, 16-bit, K-major) * V_tile(smem, MN-major, 128B swizzle).
+template <int D, bool FP16>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
+  constexpr uint32_t idesc = instr_desc(1, FP16 ? 0 : 1, 0, 1, 128, D);
+#pragma unroll
+  for (int kk = 0; kk < 128 / 16; ++kk) {
+    // 16 keys per step = 16 rows of 128 B; 64-column panels of V are 128 x 128 B apart (LBO),
+    // groups of 8 key rows are 1024 B apart (SBO).
+    const uint64_t bd = smem_desc(v_smem + kk * 16 * 128, 128 * 128, 1024, kSwizzle128B);
+    mma_f16_ts(o_tmem, p_tmem + kk * 8, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi, bool fp16) {
+  if (fp16) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+template <int D, bool INT8, bool FP16>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D, INT8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = q_full + 2;
+  uint64_t* k_empty = k_full + C::KSTAGES;
+  uint64_t* v_full = k_empty + C::KSTAGES;
+  uint64_t* v_empty = v_full + C::VSTAGES;
+  uint64_t* s_full = v_empty + C::VSTAGES;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* drain = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_done[i], 1);
+    }
+    for (int i = 0; i < C::KSTAGES; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+    for (int i = 0; i < C::VSTAGES; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // ---- work item: (m block of 256 query rows, batch, query head); heaviest causal blocks first ----
+  const int BH = p.B * p.Hq;
+  int mb = (int)(blockIdx.x / (unsigned)BH);
+  const int bh = (int)(blockIdx.x % (unsigned)BH);
+  if (p.causal) mb = p.n_mblocks - 1 - mb;
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int kvz = b * p.Hkv + h / (p.Hq / p.Hkv);
+  const int nkv = (p.N + 127) / 128;
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int row0 = mb * 256 + 128 * t;
+    n_t[t] = row0 < p.N ? (p.causal ? min(nkv, row0 / 128 + 1) : nkv) : 0;
+  }
+  const int nmax = max(n_t[0], n_t[1]);
+
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+
+  if (warp == 8) {
+    // ================================ TMA producer ================================
+    if (lane == 0) {
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_last();
+      int k_issued = 0, v_issued = 0;
+      bool ok = true;
+      for (int t = 0; t < 2; ++t) {
+        if (n_t[t] == 0) continue;
+        mbar_arrive_expect_tx(&q_full[t], C::Q_TILE);
+        for (int pn = 0; pn < C::QK_PANELS; ++pn)
+          tma_load_3d(sQ + t * C::Q_TILE + pn * C::QK_PANEL_BYTES, &tmQ, pn * C::QK_BOX_X, mb * 256 + 128 * t, bh,
+                      &q_full[t], pol_stream);
+      }
+      for (int j = 0; j < nmax && ok; ++j) {
+        const int ks = j % C::KSTAGES, vs = j % C::VSTAGES;
+        if (!(ok = mbar_wait(&k_empty[ks], ((j / C::KSTAGES) & 1) ^ 1, abort_flag, W_LOAD + 1))) break;
+        mbar_arrive_expect_tx(&k_full[ks], C::K_TILE);
+        for (int pn = 0; pn < C::QK_PANELS; ++pn)
+          tma_load_3d(sK + ks * C::K_TILE + pn * C::QK_PANEL_BYTES, &tmK, pn * C::QK_BOX_X, j * 128, kvz,
+                      &k_full[ks], pol_keep);
+        k_issued = j + 1;
+        if (!(ok = mbar_wait(&v_empty[vs], ((j / C::VSTAGES) & 1) ^ 1, abort_flag, W_LOAD + 2))) break;
+        mbar_arrive_expect_tx(&v_full[vs], C::V_TILE);
+        for (int pn = 0; pn < C::V_PANELS; ++pn)
+          tma_load_3d(sV + vs * C::V_TILE + pn * C::V_PANEL_BYTES, &tmV, pn * 64, j * 128, kvz, &v_full[vs],
+                      pol_keep);
+        v_issued = j + 1;
+      }
+      if (!ok) {
+        // Drain: every issued copy must land before the CTA's shared memory is released.
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t]) mbar_wait(&q_full[t], 0, nullptr, W_DRAIN + 1, 200000000ull);
+        for (int j = max(0, k_issued - C::KSTAGES); j < k_issued; ++j)
+          mbar_wait(&k_full[j % C::KSTAGES], (j / C::KSTAGES) & 1, nullptr, W_DRAIN + 2, 200000000ull);
+        for (int j = max(0, v_issued - C::VSTAGES); j < v_issued; ++j)
+          mbar_wait(&v_full[j % C::VSTAGES], (j / C::VSTAGES) & 1, nullptr, W_DRAIN + 3, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ================================ MMA issuer ================================
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      auto users_first = [&](int j) { return j < n_t[0] ? 0 : 1; };
+      auto users_last = [&](int j) { return j < n_t[1] ? 1 : 0; };
+      // prologue: S_t(0) for both tiles
+      if (nmax > 0) {
+        ok = mbar_wait(&k_full[0], 0, abort_flag, W_MMA + 1);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (n_t[t] == 0) continue;
+          if (!(ok = mbar_wait(&q_full[t], 0, abort_flag, W_MMA + 2))) break;
+          tc_fence_after();
+          issue_qk<D, INT8, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr);
+          mma_commit(&s_full[t]);
+          if (users_last(0) == t) mma_commit(&k_empty[0]);
+        }
+      }
+      for (int j = 0; j < nmax && ok; ++j) {
+        const int vs = j % C::VSTAGES;
+        const int ks1 = (j + 1) % C::KSTAGES;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= n_t[t]) continue;
+          if (!(ok = mbar_wait(&p_full[t], j & 1, abort_flag, W_MMA + 3))) break;
+          tc_fence_after();
+          if (users_first(j) == t) {
+            if (!(ok = mbar_wait(&v_full[vs], (j / C::VSTAGES) & 1, abort_flag, W_MMA + 4))) break;
+            tc_fence_after();
+          }
+          issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
+          mma_commit(&o_done[t]);
+          if (users_last(j) == t) mma_commit(&v_empty[vs]);
+          if (j + 1 < n_t[t]) {
+            if (users_first(j + 1) == t) {
+              if (!(ok = mbar_wait(&k_full[ks1], ((j + 1) / C::KSTAGES) & 1, abort_flag, W_MMA + 5))) break;
+              tc_fence_after();
+            }
+            issue_qk<D, INT8, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr + ks1 * C::K_TILE);
+            mma_commit(&s_full[t]);
+            if (users_last(j + 1) == t) mma_commit(&k_empty[ks1]);
+          }
+        }
+      }
+      if (!ok) {
+        // Drain: wait until every MMA issued so far has completed before TMEM is released.
+        mma_commit(drain);
+        mbar_wait(drain, 0, nullptr, W_DRAIN + 4, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================================ softmax (one row per thread) ================================
+    const int t = warp >> 2, wq = warp & 3;
+    const int nt = n_t[t];
+    const int row0 = mb * 256 + 128 * t;
+    const int row = row0 + wq * 32 + lane;
+    const uint32_t tS = tmem + C::tm_s(t) + ((uint32_t)(wq * 32) << 16);
+    const uint32_t tO = tmem + C::tm_o(t) + ((uint32_t)(wq * 32) << 16);
+    const int nblk = (p.N + 127) / 128;
+    // (an empty tile, row0 >= N, reads nothing: its sq entry does not exist)
+    const float sq_scale = (INT8 && nt > 0) ? p.sq[(size_t)bh * nblk + row0 / 128] * p.scale_log2 : p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      ok = mbar_wait(&s_full[t], j & 1, abort_flag, W_SOFTMAX + 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
+      const float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nblk + j]) : sq_scale;
+      // masks: causal diagonal tile (key > query) and the ragged last key tile (key >= N).
+      // Keys [0, lim) of this tile are visible; masked scores are left out of the max and their
+      // p is set to 0 (a select, so no -inf * 0 can arise when a quantisation scale is 0).
+      const int col0 = j * 128;
+      const bool diag = p.causal && (j == nt - 1);
+      const bool masked = diag || (col0 + 128 > p.N);
+      const int lim = (diag ? min(row + 1, p.N) : p.N) - col0;
+      float m_tile;
+      if constexpr (INT8) {
+        int mx0 = INT_MIN, mx1 = INT_MIN, mx2 = INT_MIN, mx3 = INT_MIN;
+#pragma unroll
+        for (int i = 0; i < 128; i += 4) {
+          const int* ri = reinterpret_cast<const int*>(&r[i >> 5][i & 31]);
+          mx0 = max(mx0, (!masked || i < lim) ? ri[0] : INT_MIN);
+          mx1 = max(mx1, (!masked || i + 1 < lim) ? ri[1] : INT_MIN);
+          mx2 = max(mx2, (!masked || i + 2 < lim) ? ri[2] : INT_MIN);
+          mx3 = max(mx3, (!masked || i + 3 < lim) ? ri[3] : INT_MIN);
+        }
+        m_tile = (float)max(max(mx0, mx1), max(mx2, mx3)) * sc;
+      } else {
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; i += 4) {
+          const float* ri = reinterpret_cast<const float*>(&r[i >> 5][i & 31]);
+          mx0 = fmaxf(mx0, (!masked || i < lim) ? ri[0] : -INFINITY);
+          mx1 = fmaxf(mx1, (!masked || i + 1 < lim) ? ri[1] : -INFINITY);
+          mx2 = fmaxf(mx2, (!masked || i + 2 < lim) ? ri[2] : -INFINITY);
+          mx3 = fmaxf(mx3, (!masked || i + 3 < lim) ? ri[3] : -INFINITY);
+        }
+        m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc;
+      }
+      const float m_new = fmaxf(m_run, m_tile);
+      const bool need = m_new > m_run + 8.0f;
+      const bool rescale = __any_sync(0xffffffffu, need);  // warp-uniform: TMEM ld/st are .aligned
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = ex2_approx(m_run - m_new);
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      const float neg_m = -m_run;
+      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+      for (int qtr = 0; qtr < 4; ++qtr) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float pp[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = 32 * qtr + 2 * i + e;
+            const uint32_t bits = r[col >> 5][col & 31];
+            float x;
+            if constexpr (INT8) {
+              // exact int32 -> float for |x| < 2^22 (here |x| <= 128 * 127^2): add 1.5 * 2^23 as bits
+              x = __int_as_float((int)(bits + 0x4B400000u)) - 12582912.0f;
+            } else {
+              x = __uint_as_float(bits);
+            }
+            float pv = ex2_approx(fmaf(x, sc, neg_m));
+            if (masked && col >= lim) pv = 0.f;
+            pp[e] = pv;
+          }
+          if (i & 1) { l2 += pp[0]; l3 += pp[1]; } else { l0 += pp[0]; l1 += pp[1]; }
+          pk[i] = pack2(pp[0], pp[1], FP16);
+        }
+        tmem_st16(tS + 16 * qtr, pk);
+      }
+      l_run += (l0 + l1) + (l2 + l3);
+      if (rescale && j > 0) {
+        // O holds the P V sums of tiles 0..j-1; the last of them must have landed before the
+        // rescale, and P V of tile j is issued only after this thread arrives on p_full.
+        ok = mbar_wait(&o_done[t], (j - 1) & 1, abort_flag, W_SOFTMAX + 2);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+    if (ok && nt > 0) {
+      ok = mbar_wait(&o_done[t], (nt - 1) & 1, abort_flag, W_SOFTMAX + 3);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.0f / l_run;
+        uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)bh * p.N + (size_t)row) * (D * 2);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_ld_wait(o);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, FP16);
+          if (row < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+        if (p.lse != nullptr && row < p.N) {
+          float lse = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+          if constexpr (INT8) lse += p.bias[(size_t)bh * p.N + row];
+          p.lse[(size_t)bh * p.N + row] = lse;
+        }
+      }
+    }
+    if (!ok) {
+      // make sure this thread's TMEM traffic is finished before teardown
+      tmem_st_wait();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Probe: int32 scores of selected (b, h, m_tile, n_tile) tiles through the same TMA staging
+// (FwdCfg<D, true> layouts, same tensor maps) and the same issue_qk<D, true> MMA sequence.
+// 160 threads: warps 0-3 read TMEM and write `out`, warp 4 loads and issues.
+// ------------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(160, 1)
+    probe_qk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, int B, int Hq,
+                    int Hkv, int N, const int32_t* tiles, int32_t* out) {
+  using C = FwdCfg<D, true>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + C::Q_TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::Q_TILE + C::K_TILE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int tb = tiles[4 * blockIdx.x + 0], th = tiles[4 * blockIdx.x + 1];
+  const int tm = tiles[4 * blockIdx.x + 2], tn = tiles[4 * blockIdx.x + 3];
+  const int nblk = (N + 127) / 128;
+  const bool valid = tb >= 0 && tb < B && th >= 0 && th < Hq && tm >= 0 && tm < nblk && tn >= 0 && tn < nblk;
+  int32_t* dst = out + (size_t)blockIdx.x * 128 * 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0 && valid) {
+      const int kvz = tb * Hkv + th / (Hq / Hkv);
+      mbar_arrive_expect_tx(&bars[0], C::Q_TILE + C::K_TILE);
+      for (int pn = 0; pn < C::QK_PANELS; ++pn) {
+        tma_load_3d(sQ + pn * C::QK_PANEL_BYTES, &tmQ, pn * C::QK_BOX_X, tm * 128, tb * Hq + th, &bars[0],
+                    policy_evict_first());
+        tma_load_3d(sK + pn * C::QK_PANEL_BYTES, &tmK, pn * C::QK_BOX_X, tn * 128, kvz, &bars[0],
+                    policy_evict_first());
+      }
+      if (mbar_wait(&bars[0], 0, abort_flag, W_PROBE + 1)) {
+        tc_fence_after();
+        issue_qk<D, true, false>(tmem, smem_u32(sQ), smem_u32(sK));
+      }
+      mma_commit(&bars[1]);
+    }
+    __syncwarp();
+  } else {
+    const int row = warp * 32 + lane;
+    bool ok = true;
+    if (valid) {
+      ok = mbar_wait(&bars[1], 0, abort_flag, W_PROBE + 2);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (valid && ok && !*abort_flag) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32 * c, r);
+        tmem_ld_wait(r);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)row * 128 + 32 * c);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) d4[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+      }
+    } else {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)row * 128);
+      for (int v = 0; v < 32; ++v) d4[v] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+}  // namespace tattn
