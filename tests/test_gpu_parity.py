@@ -1,8 +1,11 @@
 """GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
 
-Tolerances (element-wise, against float64 on the same bf16/fp16 input bytes):
-  bf16_exact: max |O - O_ref| <= 2e-2, mean |O - O_ref| <= 2e-3, max |lse - lse_ref| <= 1e-3
-  int8_qk:    cosine(O, O_ref) >= 0.999 and max |O - O_ref| <= 5e-2 against exact attention,
+Tolerances (element-wise, against float64 on the same bf16/fp16 input bytes).  The output error is
+e = |O - O_ref| / max(1, |O_ref|): absolute for |O_ref| <= 1, relative above.  The output is stored in
+bf16, whose rounding alone is 2^-9 relative, so an absolute 2e-2 bound cannot hold for outputs above
+~10 in magnitude (the workload with x10 outlier channels in V reaches |O| ~ 20-40).
+  bf16_exact: max e <= 2e-2, mean e <= 2e-3, max |lse - lse_ref| <= 1e-3
+  int8_qk:    cosine(O, O_ref) >= 0.999 and max e <= 5e-2 against exact attention,
               the bf16_exact bounds against the INT8 emulation (same quantised scores),
               max |lse - lse_ref| <= 5e-2
   pre-pass:   q8, k8, sq, sk, kmean bit-exact; lse_bias within 1e-4 (+1e-4 relative)
@@ -46,8 +49,12 @@ def gpu_fwd(ta, q, k, v, causal, mode):
     return _np(o), l.cpu().numpy().astype(np.float64)
 
 
+def scaled_err(o, O):
+    return np.abs(o - O) / np.maximum(1.0, np.abs(O))
+
+
 def assert_bf16(o, l, O, L, what=""):
-    err = np.abs(o - O)
+    err = scaled_err(o, O)
     assert np.isfinite(o).all(), what
     assert err.max() <= BF16_MAX, f"{what}: max abs err {err.max():.3e}"
     assert err.mean() <= BF16_MEAN, f"{what}: mean abs err {err.mean():.3e}"
@@ -62,7 +69,7 @@ def cosine(a, b):
 def assert_int8(o, l, O, L, what=""):
     assert np.isfinite(o).all(), what
     c = cosine(o, O)
-    err = np.abs(o - O).max()
+    err = scaled_err(o, O).max()
     assert c >= INT8_COS, f"{what}: cosine {c:.6f}"
     assert err <= INT8_MAX, f"{what}: max abs err {err:.3e}"
     assert np.abs(l - L).max() <= INT8_LSE, f"{what}: lse err {np.abs(l - L).max():.3e}"
@@ -191,7 +198,7 @@ def test_full_size_sampled_rows(ta, cfg, mode):
             Oe, Le = emulated(qs, ks, vs, w.causal, w.scale, rows=rows)
             assert_bf16(og, lg, Oe, Le, f"cfg{cfg} b{b} h{h} vs emulation")
             assert np.abs(lg - L).max() <= INT8_LSE
-            assert np.abs(og - O).max() <= INT8_MAX
+            assert scaled_err(og, O).max() <= INT8_MAX
             o_all.append(og.reshape(-1))
             O_all.append(O.reshape(-1))
     if mode == "int8_qk":
@@ -220,7 +227,7 @@ def test_large_scores_exercise_rescaling(ta, mode):
         assert_bf16(o, l, O, L)
     else:
         Oe, Le = emulated(q, k, v, False, w.scale)
-        assert np.abs(o - Oe).max() <= BF16_MAX and np.abs(l - Le).max() <= INT8_LSE
+        assert scaled_err(o, Oe).max() <= BF16_MAX and np.abs(l - Le).max() <= INT8_LSE
 
 
 def test_deterministic_and_gqa_equals_expanded_mha(ta):
