@@ -63,6 +63,14 @@ struct FwdCfg {
   static constexpr int V_PANEL_BYTES = BN * 128;
   static constexpr int V_TILE = BN * D * 2;
   static constexpr int PV_STEPS = BN / 16;
+  // of every 16 score columns, how many take exp2_poly (FMA pipe) instead of MUFU ex2
+#ifndef TATTN_POLY_BF16
+#define TATTN_POLY_BF16 0
+#endif
+#ifndef TATTN_POLY_INT8
+#define TATTN_POLY_INT8 0
+#endif
+  static constexpr int POLY_PER_16 = INT8 ? TATTN_POLY_INT8 : TATTN_POLY_BF16;
   static constexpr int KSTAGES = (D == 128 && !INT8) ? 2 : 4;
   static constexpr int VSTAGES = (D == 128) ? (INT8 ? 3 : 2) : 4;
   static constexpr int OFF_Q = 0;
@@ -114,6 +122,23 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
     const uint64_t bd = smem_desc(v_smem + kk * 16 * 128, 128 * 128, 1024, kSwizzle128B);
     mma_f16_ts(o_tmem, p_tmem + kk * 8, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
+}
+
+// 2^x on the FMA pipe (offloads the MUFU unit, which does one ex2 per score).  Range reduction
+// 2^x = 2^n * 2^f with n = rint(x), f in [-1/2, 1/2] (Cody & Waite), then a degree-3 minimax
+// polynomial for 2^f fitted with the Remez algorithm by tiled_attention_22_b200/exp2_fit.py
+// (max relative error 7.5e-5 in float32 FMA arithmetic, below the 2^-9 rounding of 16-bit P).
+// x is clamped at -125 so that adding n to the exponent field never leaves the normal range;
+// softmax arguments here are <= 8 (lazy rescale), so there is no overflow side.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;  // 1.5 * 2^23: rint(x) lands in the low mantissa bits of t
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
+  p = fmaf(p, f, 6.932609677e-01f);
+  p = fmaf(p, f, 9.999280572e-01f);
+  // the low 9 bits of t's pattern above the integer are zero, so (bits(t) << 23) == n << 23
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool fp16) {
@@ -371,7 +396,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             } else {
               x = __uint_as_float(bits);
             }
-            float pv = ex2_approx(fmaf(x, sc, neg_m));
+            const float arg = fmaf(x, sc, neg_m);
+            float pv;
+            if ((col & 15) >= 16 - C::POLY_PER_16)
+              pv = exp2_poly(arg);
+            else
+              pv = ex2_approx(arg);
             if (masked && col >= lim) pv = 0.f;
             pp[e] = pv;
           }
