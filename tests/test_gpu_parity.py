@@ -316,3 +316,16 @@ def test_bounded_wait_reports_timeout_and_context_survives(ta):
     o, l = gpu_fwd(ta, q, k, v, False, "bf16_exact")
     O, L = oracle.attention(q, k, v, w.scale, False)
     assert_bf16(o, l, O, L)
+
+
+@pytest.mark.parametrize("use_poly", [True, False])
+def test_kernel_exp2_against_cuda_exp2f(ta, use_poly):
+    """The softmax's exp2 routines against CUDA's exp2f on the softmax argument range.  The
+    polynomial's bound is its Remez fit (7.5e-5 relative) plus float32 rounding; ex2.approx is
+    documented to about 2 ulp."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, -1e-7, 7.999])]).cuda()
+    y = ta.attn_test_exp2(x, use_poly)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel <= (8e-5 if use_poly else 1e-6), rel
+    assert torch.isfinite(y).all()

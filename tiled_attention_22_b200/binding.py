@@ -42,6 +42,7 @@ _SIGNATURES = {
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_last_cuda_error": (ctypes.c_char_p, []),
     "attn_test_wait_timeout": (_i, [_i, _vp]),
+    "attn_test_exp2": (_i, [_vp, _vp, _i, _i, _vp]),
 }
 
 _lib = None
@@ -220,3 +221,11 @@ def attn_error_string(code: int) -> str:
 
 def attn_test_wait_timeout(limit_us: int, stream=None) -> None:
     _check(load_library().attn_test_wait_timeout(int(limit_us), _stream(stream)), "attn_test_wait_timeout")
+
+
+def attn_test_exp2(x, use_poly: bool, stream=None):
+    """Apply the kernel's exp2 routine (polynomial or MUFU) to a float32 CUDA tensor."""
+    y = torch.empty_like(x)
+    _check(load_library().attn_test_exp2(_ptr(x), _ptr(y), x.numel(), int(bool(use_poly)), _stream(stream)),
+           "attn_test_exp2")
+    return y

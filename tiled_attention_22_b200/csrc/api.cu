@@ -99,6 +99,16 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
   if ((rc = make_map(&tv, v, v_dt, 2, D, p.N, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
   auto kern = attn_fwd_kernel<D, INT8, FP16>;
   TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+  // The kernel moves registers between warpgroups with setmaxnreg; the increase only completes if
+  // the registers the CTA is launched with cover the split.  Refuse to launch otherwise.
+  cudaFuncAttributes attr;
+  TATTN_CUDA(cudaFuncGetAttributes(&attr, kern));
+  if ((long long)attr.numRegs * kFwdThreads < 128LL * (2 * kRegsSoftmax + kRegsProducer) ||
+      attr.maxThreadsPerBlock < kFwdThreads) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "fused kernel built with %d registers/thread: too few for its register split", attr.numRegs);
+    return ATTN_ERR_LAUNCH;
+  }
   const long long grid = (long long)p.n_mblocks * p.B * p.Hq;
   kern<<<(unsigned)grid, kFwdThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   TATTN_CUDA(cudaGetLastError());
@@ -121,6 +131,13 @@ FwdParams make_params(int B, int Hq, int Hkv, int N, int causal, float scale, vo
   p.N = N;
   p.causal = causal;
   p.n_mblocks = (N + 255) / 256;
+  // Scheduling sections: kv heads whose K and V (16-bit, the larger case) take at most ~32 MB,
+  // a quarter of the 126 MB L2.
+  const long long kv_bytes = 2LL * N * 128 * 2;
+  long long sec = (32LL << 20) / (kv_bytes > 0 ? kv_bytes : 1);
+  if (sec < 1) sec = 1;
+  if (sec > (long long)B * Hkv) sec = (long long)B * Hkv;
+  p.sec_kv = (int)sec;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = o;
   p.lse = lse;
@@ -208,6 +225,11 @@ int fwd_int8_quantized(const int8_t* q8, const float* sq, const int8_t* k8, cons
   p.sk = sk;
   p.bias = bias;
   return launch_fwd<true>(q8, k8, v, d, dtype, p, stream);
+}
+
+__global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int use_poly) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = use_poly ? exp2_poly(x[i]) : ex2_approx(x[i]);
 }
 
 __global__ void wait_forever_probe_kernel(unsigned long long limit_ns) {
@@ -346,6 +368,15 @@ int attn_check_status(void) {
 int attn_test_wait_timeout(int limit_us, void* stream) {
   if (limit_us < 1 || limit_us > 1000000) return ATTN_ERR_ARG;
   wait_forever_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((unsigned long long)limit_us * 1000ull);
+  TATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
+// Test hook: the fused kernel's exp2 routines applied to an array (1 = FMA-pipe polynomial,
+// 0 = MUFU ex2.approx), so tests can compare them with CUDA's exp2f.
+int attn_test_exp2(const float* x, float* y, int n, int use_poly, void* stream) {
+  if (!x || !y || n < 1) return ATTN_ERR_ARG;
+  exp2_eval_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, use_poly);
   TATTN_CUDA(cudaGetLastError());
   return ATTN_OK;
 }

@@ -11,11 +11,14 @@
 // article, section 技术方案), and P V stays in 16-bit floating point.
 //
 // B200 design (not the pages'; their kernels target Ampere/Ada/Hopper):
-//   * CTA = 2 query tiles of 128 rows, 320 threads in four roles:
+//   * CTA = 2 query tiles of 128 rows, 384 threads in four roles:
 //       warps 0-3  softmax for query tile 0 (thread = one row; TMEM lanes 0..127)
 //       warps 4-7  softmax for query tile 1
 //       warp  8    TMA producer: Q tiles once, then K and V tiles through separate mbarrier rings
 //       warp  9    MMA issuer (one thread): tcgen05.mma S = Q K^T into TMEM, O += P V from TMEM
+//       warps 10-11 idle (they complete the producer warpgroup for the register split)
+//     setmaxnreg moves registers from the producer warpgroup (56/thread) to the softmax
+//     warpgroups (224/thread).
 //   * TMEM (512 columns): S/P of tile t at column 128 t; O of tile t at column 256 + t D.
 //     P (16-bit) is written over the first 64 columns of S and consumed as the A operand of P V
 //     straight from TMEM, so P never touches shared memory.
@@ -38,6 +41,7 @@ namespace tattn {
 struct FwdParams {
   int B, Hq, Hkv, N, causal;
   int n_mblocks;          // ceil(N / 256)
+  int sec_kv;             // kv heads per scheduling section (K/V of a section stay in L2)
   float scale_log2;       // scale * log2(e)
   void* o;                // [B, Hq, N, D] 16-bit
   float* lse;             // [B, Hq, N] or null
@@ -89,7 +93,12 @@ struct FwdCfg {
   static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 };
 
-constexpr int kFwdThreads = 320;
+// 12 warps: two softmax warpgroups and one producer warpgroup (TMA warp, MMA warp, 2 idle).
+constexpr int kFwdThreads = 384;
+constexpr int kLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
+constexpr int kRegsSoftmax = 208;  // per thread, softmax warpgroups
+constexpr int kRegsProducer = 88;  // per thread, producer warpgroup
+static_assert(128 * (2 * kRegsSoftmax + kRegsProducer) <= kFwdThreads * kLaunchRegs, "register split");
 
 // Wait-site ids recorded with a timeout (role * 16 + barrier kind).
 enum : int { W_LOAD = 0x10, W_MMA = 0x20, W_SOFTMAX = 0x30, W_DRAIN = 0x40, W_PROBE = 0x50 };
@@ -150,6 +159,122 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool fp16) {
   return *reinterpret_cast<uint32_t*>(&b);
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Packed pair arithmetic (sm_100 f32x2): one instruction for two FP32 lanes.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
+        "l"(*reinterpret_cast<uint64_t*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
+// One online-softmax step of one score row (this thread's row of the 128 x 128 tile in TMEM):
+//   x = scores of the tile (fp32, or the int32 INT8 scores as 2^23*1.5 + acc, exact);
+//   m_tile = max x * sc; the running max moves only when it grows by more than 8 (log2 units);
+//   p = 2^(x*sc - m) rounded to 16 bits and stored over the first 64 columns of S (P V's A
+//   operand); l accumulates the unrounded p; O is rescaled in TMEM when the max moved.
+// MASKED: keys at tile columns >= lim are invisible (causal diagonal or past N): their x is
+// -inf, so p = 2^-inf = 0 exactly (these tiles use MUFU ex2 for every column).
+template <int D, bool INT8, bool FP16, bool MASKED>
+__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc, int lim, int j, float& m_run,
+                                             float& l_run, uint64_t* o_done_t, volatile int* abort_flag) {
+  using C = FwdCfg<D, INT8>;
+  uint32_t r[4][32];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
+  float x[128];
+#pragma unroll
+  for (int i = 0; i < 128; ++i) {
+    const uint32_t bits = r[i >> 5][i & 31];
+    // INT8: exact int32 -> float for |acc| < 2^22 (here |acc| <= 128 * 127^2): x = 1.5*2^23 + acc
+    x[i] = INT8 ? __uint_as_float(bits + 0x4B400000u) : __uint_as_float(bits);
+    if (MASKED && i >= lim) x[i] = -INFINITY;
+  }
+  float mc[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float m = x[32 * c];
+#pragma unroll
+    for (int k = 1; k < 31; k += 2) m = max3f(m, x[32 * c + k], x[32 * c + k + 1]);
+    mc[c] = fmaxf(m, x[32 * c + 31]);
+  }
+  const float mx = max3f(mc[0], mc[1], fmaxf(mc[2], mc[3]));
+  const float m_tile = INT8 ? (mx - 12582912.0f) * sc : mx * sc;
+  // Each row decides for itself whether its running max moves (so its rounding never depends on
+  // other rows); the TMEM rescale of O below is warp-uniform (.aligned), and rows that keep their
+  // max multiply by exactly 1.
+  const float m_new = fmaxf(m_run, m_tile);
+  const bool need = m_new > m_run + 8.0f;
+  const bool rescale = __any_sync(0xffffffffu, need);
+  float alpha = 1.f;
+  if (need) {
+    alpha = ex2_approx(m_run - m_new);
+    l_run *= alpha;
+    m_run = m_new;
+  }
+  // exponent argument x*sc + cst; INT8 folds the 1.5*2^23 offset into the constant
+  const float cst = INT8 ? -fmaf(12582912.0f, sc, m_run) : -m_run;
+  const float2 sc2 = make_float2(sc, sc), cst2 = make_float2(cst, cst);
+  float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int qtr = 0; qtr < 4; ++qtr) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int col = 32 * qtr + 2 * i;
+      const float2 a = ffma2(make_float2(x[col], x[col + 1]), sc2, cst2);
+      float p0, p1;
+      if (!MASKED && (col & 15) >= 16 - C::POLY_PER_16) {
+        p0 = exp2_poly(a.x);
+        p1 = exp2_poly(a.y);
+      } else {
+        p0 = ex2_approx(a.x);
+        p1 = ex2_approx(a.y);
+      }
+      if (i & 1)
+        ls1 = fadd2(ls1, make_float2(p0, p1));
+      else
+        ls0 = fadd2(ls0, make_float2(p0, p1));
+      pk[i] = pack2(p0, p1, FP16);
+    }
+    tmem_st16(tS + 16 * qtr, pk);
+  }
+  l_run += (ls0.x + ls0.y) + (ls1.x + ls1.y);
+  if (rescale && j > 0) {
+    // O holds the P V sums of tiles 0..j-1; the last of them must have landed before the rescale,
+    // and P V of tile j is issued only after this thread arrives on p_full.
+    bool ok = mbar_wait(o_done_t, (j - 1) & 1, abort_flag, W_SOFTMAX + 2);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return false;
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + 32 * c, o);
+      tmem_ld_wait(o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+      tmem_st32(tO + 32 * c, o);
+    }
+  }
+  return true;
+}
+
 template <int D, bool INT8, bool FP16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -199,13 +324,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // ---- work item: (m block of 256 query rows, batch, query head); heaviest causal blocks first ----
-  const int BH = p.B * p.Hq;
-  int mb = (int)(blockIdx.x / (unsigned)BH);
-  const int bh = (int)(blockIdx.x % (unsigned)BH);
-  if (p.causal) mb = p.n_mblocks - 1 - mb;
-  const int b = bh / p.Hq, h = bh % p.Hq;
-  const int kvz = b * p.Hkv + h / (p.Hq / p.Hkv);
+  // ---- work item: (m block of 256 query rows, batch, query head) ----
+  // CTAs are ordered in sections of sec_kv consecutive (batch, kv head) pairs, sized on the host
+  // so that a section's K and V fit comfortably in L2: all query heads and m blocks of a section
+  // run close together and share those K/V tiles through L2.  Inside a section, m blocks go
+  // heaviest first under causal masking (longest rows start first), query heads fastest.
+  const int G = p.Hq / p.Hkv;
+  const int n_bkv = p.B * p.Hkv;
+  const int per_sec = p.sec_kv * G * p.n_mblocks;
+  const int sec = (int)(blockIdx.x / (unsigned)per_sec);
+  const int kv0 = sec * p.sec_kv;
+  const int nkv_sec = min(p.sec_kv, n_bkv - kv0);
+  const int rr = (int)blockIdx.x - sec * per_sec;
+  const int mb_rank = rr / (nkv_sec * G);
+  const int within = rr - mb_rank * (nkv_sec * G);
+  const int kvz = kv0 + within / G;  // b * Hkv + kv head
+  const int mb = p.causal ? p.n_mblocks - 1 - mb_rank : mb_rank;
+  const int b = kvz / p.Hkv;
+  const int h = (kvz - b * p.Hkv) * G + within % G;
+  const int bh = b * p.Hq + h;
   const int nkv = (p.N + 127) / 128;
   int n_t[2];
 #pragma unroll
@@ -219,6 +356,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
 
+  if (warp >= 8) {
+    regs_decrease<kRegsProducer>();
   if (warp == 8) {
     // ================================ TMA producer ================================
     if (lane == 0) {
@@ -310,7 +449,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     __syncwarp();
+  }  // warps 10-11: nothing to do
   } else {
+    regs_increase<kRegsSoftmax>();
     // ================================ softmax (one row per thread) ================================
     const int t = warp >> 2, wq = warp & 3;
     const int nt = n_t[t];
@@ -328,106 +469,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t r[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
-      const float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nblk + j]) : sq_scale;
-      // masks: causal diagonal tile (key > query) and the ragged last key tile (key >= N).
-      // Keys [0, lim) of this tile are visible; masked scores are left out of the max and their
-      // p is set to 0 (a select, so no -inf * 0 can arise when a quantisation scale is 0).
+      float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nblk + j]) : sq_scale;
+      if constexpr (INT8) sc = fmaxf(sc, 1e-30f);  // a zero block: keep -inf * sc = -inf for masks
+      // causal diagonal tile (key > query) and the ragged last key tile (key >= N) are masked;
+      // keys [0, lim) of the tile are visible
       const int col0 = j * 128;
       const bool diag = p.causal && (j == nt - 1);
-      const bool masked = diag || (col0 + 128 > p.N);
-      const int lim = (diag ? min(row + 1, p.N) : p.N) - col0;
-      float m_tile;
-      if constexpr (INT8) {
-        int mx0 = INT_MIN, mx1 = INT_MIN, mx2 = INT_MIN, mx3 = INT_MIN;
-#pragma unroll
-        for (int i = 0; i < 128; i += 4) {
-          const int* ri = reinterpret_cast<const int*>(&r[i >> 5][i & 31]);
-          mx0 = max(mx0, (!masked || i < lim) ? ri[0] : INT_MIN);
-          mx1 = max(mx1, (!masked || i + 1 < lim) ? ri[1] : INT_MIN);
-          mx2 = max(mx2, (!masked || i + 2 < lim) ? ri[2] : INT_MIN);
-          mx3 = max(mx3, (!masked || i + 3 < lim) ? ri[3] : INT_MIN);
-        }
-        m_tile = (float)max(max(mx0, mx1), max(mx2, mx3)) * sc;
+      if (diag || (col0 + 128 > p.N)) {
+        const int lim = (diag ? min(row + 1, p.N) : p.N) - col0;
+        ok = softmax_step<D, INT8, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
       } else {
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 128; i += 4) {
-          const float* ri = reinterpret_cast<const float*>(&r[i >> 5][i & 31]);
-          mx0 = fmaxf(mx0, (!masked || i < lim) ? ri[0] : -INFINITY);
-          mx1 = fmaxf(mx1, (!masked || i + 1 < lim) ? ri[1] : -INFINITY);
-          mx2 = fmaxf(mx2, (!masked || i + 2 < lim) ? ri[2] : -INFINITY);
-          mx3 = fmaxf(mx3, (!masked || i + 3 < lim) ? ri[3] : -INFINITY);
-        }
-        m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc;
+        ok = softmax_step<D, INT8, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
       }
-      // Each row decides for itself whether its running max moves (so its rounding never depends
-      // on other rows); the TMEM rescale of O below is warp-uniform (.aligned), and rows that keep
-      // their max multiply by exactly 1.
-      const float m_new = fmaxf(m_run, m_tile);
-      const bool need = m_new > m_run + 8.0f;
-      const bool rescale = __any_sync(0xffffffffu, need);
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2_approx(m_run - m_new);
-        l_run *= alpha;
-        m_run = m_new;
-      }
-      const float neg_m = -m_run;
-      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-#pragma unroll
-      for (int qtr = 0; qtr < 4; ++qtr) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float pp[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 32 * qtr + 2 * i + e;
-            const uint32_t bits = r[col >> 5][col & 31];
-            float x;
-            if constexpr (INT8) {
-              // exact int32 -> float for |x| < 2^22 (here |x| <= 128 * 127^2): add 1.5 * 2^23 as bits
-              x = __int_as_float((int)(bits + 0x4B400000u)) - 12582912.0f;
-            } else {
-              x = __uint_as_float(bits);
-            }
-            const float arg = fmaf(x, sc, neg_m);
-            float pv;
-            if ((col & 15) >= 16 - C::POLY_PER_16)
-              pv = exp2_poly(arg);
-            else
-              pv = ex2_approx(arg);
-            if (masked && col >= lim) pv = 0.f;
-            pp[e] = pv;
-          }
-          if (i & 1) { l2 += pp[0]; l3 += pp[1]; } else { l0 += pp[0]; l1 += pp[1]; }
-          pk[i] = pack2(pp[0], pp[1], FP16);
-        }
-        tmem_st16(tS + 16 * qtr, pk);
-      }
-      l_run += (l0 + l1) + (l2 + l3);
-      if (rescale && j > 0) {
-        // O holds the P V sums of tiles 0..j-1; the last of them must have landed before the
-        // rescale, and P V of tile j is issued only after this thread arrives on p_full.
-        ok = mbar_wait(&o_done[t], (j - 1) & 1, abort_flag, W_SOFTMAX + 2);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_ld_wait(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + 32 * c, o);
-        }
-      }
+      if (!ok) break;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
