@@ -115,6 +115,29 @@ int attn_quant_smooth_k(const void* q, const void* k, int B, int Hq, int Hkv, in
 size_t attn_quant_scratch_bytes(int B, int Hkv, int N, int d);
 
 /*
+ * attn_quant_smooth_k_noalloc - the same pre-pass as attn_quant_smooth_k, for callers that cannot
+ * allocate device memory: code that runs under another owner's memory pool that hands out no
+ * extra device buffers, or a latency-bound loop that cannot afford cudaMalloc (which may
+ * synchronise the whole device).  (The pages have no counterpart: this is an interface choice.)
+ *
+ *   Arguments and results are those of attn_quant_smooth_k without scratch / scratch_bytes: the
+ *   caller still passes q, k and every output buffer.  The float64 K-mean partials go to an
+ *   8 MiB array built into the library; each GPU that loads the library keeps its copy until the
+ *   process exits.  Sizes are limited to B*Hkv*ceil(N/128)*d <= 1048576 (e.g. B=1, Hkv=8,
+ *   N=131072, d=128); larger sizes return ATTN_ERR_WORKSPACE before launching (text in
+ *   attn_last_cuda_error) and need attn_quant_smooth_k.
+ *   The first call on each device looks up the array's device address (with that device
+ *   current) and caches it; make that first call before any stream capture on that device.
+ *   The call itself allocates nothing.  All calls on a device share the one array, and it keeps
+ *   the previous call's contents (every entry a call reads is written by the same call first):
+ *   calls whose kernels overlap on the GPU (different streams, no ordering) race on it, so order
+ *   them, for example by issuing them on one stream.
+ */
+int attn_quant_smooth_k_noalloc(const void* q, const void* k, int B, int Hq, int Hkv, int N, int d,
+                                int dtype, float scale, int8_t* q8, float* sq, int8_t* k8,
+                                float* sk, float* kmean, float* lse_bias, void* stream);
+
+/*
  * attn_fwd_int8_quantized - the fused INT8 attention kernel alone, on the
  * outputs of attn_quant_smooth_k (q8, sq, k8, sk, lse_bias; all device).
  * v, o and lse as in attn_fwd.  lse_bias may be NULL only when lse is NULL.

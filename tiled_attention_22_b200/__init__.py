@@ -21,6 +21,7 @@ from .binding import (  # noqa: F401
     attn_probe_qk_int32,
     attn_quant_scratch_bytes,
     attn_quant_smooth_k,
+    attn_quant_smooth_k_noalloc,
     attn_test_exp2,
     attn_test_wait_timeout,
     attn_workspace_bytes,

@@ -34,6 +34,7 @@ _SIGNATURES = {
     "attn_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_quant_smooth_k": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "attn_quant_scratch_bytes": (_sz, [_i, _i, _i, _i]),
+    "attn_quant_smooth_k_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "attn_fwd_int8_quantized": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_probe_qk_int32": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp]),
     "attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i,
@@ -164,6 +165,32 @@ def attn_quant_smooth_k(q, k, scale=None, scratch=None, stream=None, out=None):
                                  _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]), _ptr(out["kmean"]),
                                  _ptr(out["lse_bias"]), _ptr(scratch), scratch.numel(), _stream(stream))
     _check(rc, "attn_quant_smooth_k")
+    return out
+
+
+def attn_quant_smooth_k_noalloc(q, k, scale=None, out=None, stream=None):
+    """The pre-pass without caller scratch: its float64 K-mean partials use the library's built-in
+    8 MiB array (for callers that cannot allocate device memory).  Output buffers are still the
+    caller's; ``out`` may supply them (else they are allocated here with torch)."""
+    lib = load_library()
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    _shape(q, k, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    T = (N + 127) // 128
+    dev = q.device
+    out = out or dict(
+        q8=torch.empty((B, Hq, N, d), device=dev, dtype=torch.int8),
+        sq=torch.empty((B, Hq, T), device=dev, dtype=torch.float32),
+        k8=torch.empty((B, Hkv, N, d), device=dev, dtype=torch.int8),
+        sk=torch.empty((B, Hkv, T), device=dev, dtype=torch.float32),
+        kmean=torch.empty((B, Hkv, d), device=dev, dtype=torch.float32),
+        lse_bias=torch.empty((B, Hq, N), device=dev, dtype=torch.float32),
+    )
+    rc = lib.attn_quant_smooth_k_noalloc(_ptr(q), _ptr(k), B, Hq, Hkv, N, d, DTYPES[q.dtype], scale,
+                                         _ptr(out["q8"]), _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]),
+                                         _ptr(out["kmean"]), _ptr(out["lse_bias"]), _stream(stream))
+    _check(rc, "attn_quant_smooth_k_noalloc")
     return out
 
 

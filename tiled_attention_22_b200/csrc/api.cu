@@ -245,6 +245,40 @@ __global__ void wait_forever_probe_kernel(unsigned long long limit_ns) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, 0x7f, limit_ns);
 }
 
+// ------------------------------------------------------------------------------------------------
+// Allocation-free pre-pass.  The only device memory attn_quant_smooth_k needs beyond its inputs and
+// outputs is the float64 block partials of the K mean; this variant keeps them in a fixed array
+// that lives in the library itself, so a caller that cannot allocate device memory still gets the
+// same pre-pass.  The array is file-scope and holds up to kStaticScratchBytes; every GPU that loads
+// the library holds its own copy until the process exits.  Its host-side name is only a stand-in,
+// so its device address is looked up once per device (cudaGetSymbolAddress, with that device
+// current) and cached; kernels are given that address.
+// ------------------------------------------------------------------------------------------------
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB = 1 Mi float64 partials
+static __device__ __align__(256) double g_static_kmean_scratch[kStaticScratchBytes / sizeof(double)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+int static_scratch_address(double** out) {
+  int dev = -1;
+  TATTN_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "device ordinal %d out of range", dev);
+    return ATTN_ERR_LAUNCH;
+  }
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (g_static_scratch_addr[dev] == nullptr) {
+    void* addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_static_kmean_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static K-mean scratch)");
+    g_static_scratch_addr[dev] = addr;
+  }
+  *out = static_cast<double*>(g_static_scratch_addr[dev]);
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -275,6 +309,32 @@ int attn_quant_smooth_k(const void* q, const void* k, int B, int Hq, int Hkv, in
   if (!aligned16(scratch)) return ATTN_ERR_ALIGN;
   return launch_prepass(q, k, B, Hq, Hkv, N, d, dtype, scale, q8, sq, k8, sk, kmean, lse_bias,
                         static_cast<double*>(scratch), static_cast<cudaStream_t>(stream));
+}
+
+int attn_quant_smooth_k_noalloc(const void* q, const void* k, int B, int Hq, int Hkv, int N, int d, int dtype,
+                                float scale, int8_t* q8, float* sq, int8_t* k8, float* sk, float* kmean,
+                                float* lse_bias, void* stream) {
+  if (!q || !k || !q8 || !sq || !k8 || !sk || !kmean || !lse_bias) return ATTN_ERR_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_ARG;
+  int rc = check_shape(B, Hq, Hkv, N, d);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8) || !aligned16(kmean) || !aligned16(sq) ||
+      !aligned16(sk) || !aligned16(lse_bias))
+    return ATTN_ERR_ALIGN;
+  const size_t need = scratch_bytes(B, Hkv, N, d);
+  if (need > kStaticScratchBytes) {
+    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                  "these sizes need %zu bytes of K-mean scratch; the built-in scratch holds %zu "
+                  "(B*Hkv*ceil(N/128)*d <= %zu); use attn_quant_smooth_k with caller scratch",
+                  need, kStaticScratchBytes, kStaticScratchBytes / sizeof(double));
+    return ATTN_ERR_WORKSPACE;
+  }
+  double* part = nullptr;
+  if ((rc = static_scratch_address(&part))) return rc;
+  // The partials are written in full before they are read, so nothing has to be cleared.
+  return launch_prepass(q, k, B, Hq, Hkv, N, d, dtype, scale, q8, sq, k8, sk, kmean, lse_bias, part,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd_int8_quantized(const int8_t* q8, const float* sq, const int8_t* k8, const float* sk,
