@@ -227,9 +227,10 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
     l_run *= alpha;
     m_run = m_new;
   }
-  // exponent argument x*sc + cst; INT8 folds the 1.5*2^23 offset into the constant
-  const float cst = INT8 ? -fmaf(12582912.0f, sc, m_run) : -m_run;
-  const float2 sc2 = make_float2(sc, sc), cst2 = make_float2(cst, cst);
+  // exponent argument (x - off) * sc - m, off = 1.5*2^23 for INT8 (removed exactly by the add;
+  // folding it into the constant would round off*sc + m per tile, shifting whole tiles)
+  const float2 sc2 = make_float2(sc, sc), cst2 = make_float2(-m_run, -m_run);
+  const float2 off2 = make_float2(-12582912.0f, -12582912.0f);
   float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int qtr = 0; qtr < 4; ++qtr) {
@@ -237,7 +238,9 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int col = 32 * qtr + 2 * i;
-      const float2 a = ffma2(make_float2(x[col], x[col + 1]), sc2, cst2);
+      float2 xv = make_float2(x[col], x[col + 1]);
+      if constexpr (INT8) xv = fadd2(xv, off2);
+      const float2 a = ffma2(xv, sc2, cst2);
       float p0, p1;
       if (!MASKED && (col & 15) >= 16 - C::POLY_PER_16) {
         p0 = exp2_poly(a.x);
