@@ -86,9 +86,15 @@ CUtensorMapSwizzle swizzle_for(int row_bytes) {
 }
 
 // ----------------------------------------- fused kernel launch ------------------------------------
+#ifndef TATTN_SPLIT
+#define TATTN_SPLIT 0
+#endif
+
 template <int D, bool INT8, bool FP16>
 int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p, cudaStream_t stream) {
   using C = FwdCfg<D, INT8>;
+  constexpr bool SPLIT = TATTN_SPLIT != 0;
+  using R = FwdRoles<SPLIT>;
   CUtensorMap tq, tk, tv;
   const CUtensorMapDataType qk_dt =
       INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : (FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
@@ -97,20 +103,21 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
   if ((rc = make_map(&tq, q, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hq, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
   if ((rc = make_map(&tk, k, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hkv, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
   if ((rc = make_map(&tv, v, v_dt, 2, D, p.N, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-  auto kern = attn_fwd_kernel<D, INT8, FP16>;
+  auto kern = attn_fwd_kernel<D, INT8, FP16, SPLIT>;
   TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
   // The kernel moves registers between warpgroups with setmaxnreg; the increase only completes if
   // the registers the CTA is launched with cover the split.  Refuse to launch otherwise.
   cudaFuncAttributes attr;
   TATTN_CUDA(cudaFuncGetAttributes(&attr, kern));
-  if ((long long)attr.numRegs * kFwdThreads < 128LL * (2 * kRegsSoftmax + kRegsProducer) ||
-      attr.maxThreadsPerBlock < kFwdThreads) {
+  if ((long long)attr.numRegs * R::kThreads <
+          128LL * (R::kSoftmaxWarps / 4 * R::kRegsSoftmax + R::kRegsProducer) ||
+      attr.maxThreadsPerBlock < R::kThreads) {
     std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
                   "fused kernel built with %d registers/thread: too few for its register split", attr.numRegs);
     return ATTN_ERR_LAUNCH;
   }
   const long long grid = (long long)p.n_mblocks * p.B * p.Hq;
-  kern<<<(unsigned)grid, kFwdThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  kern<<<(unsigned)grid, R::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   TATTN_CUDA(cudaGetLastError());
   return ATTN_OK;
 }
@@ -131,10 +138,13 @@ FwdParams make_params(int B, int Hq, int Hkv, int N, int causal, float scale, vo
   p.N = N;
   p.causal = causal;
   p.n_mblocks = (N + 255) / 256;
-  // Scheduling sections: kv heads whose K and V (16-bit, the larger case) take at most ~32 MB,
-  // a quarter of the 126 MB L2.
+  // Scheduling sections: kv heads whose K and V (16-bit, d=128, the larger case) take at most
+  // TATTN_L2_SECTION_MB (a quarter of the 126 MB L2 by default).
+#ifndef TATTN_L2_SECTION_MB
+#define TATTN_L2_SECTION_MB 32
+#endif
   const long long kv_bytes = 2LL * N * 128 * 2;
-  long long sec = (32LL << 20) / (kv_bytes > 0 ? kv_bytes : 1);
+  long long sec = ((long long)TATTN_L2_SECTION_MB << 20) / (kv_bytes > 0 ? kv_bytes : 1);
   if (sec < 1) sec = 1;
   if (sec > (long long)B * Hkv) sec = (long long)B * Hkv;
   p.sec_kv = (int)sec;
@@ -191,12 +201,14 @@ int launch_prepass(const void* q, const void* k, int B, int Hq, int Hkv, int N, 
   const auto* k16 = static_cast<const uint16_t*>(k);
   const auto* q16 = static_cast<const uint16_t*>(q);
   {
-    const long long threads = (long long)BG * T * (d / 8);
-    const unsigned blocks = (unsigned)((threads + 127) / 128);
-    if (fp16)
-      kmean_partial_kernel<true><<<blocks, 128, 0, stream>>>(k16, BG, N, d, part);
-    else
-      kmean_partial_kernel<false><<<blocks, 128, 0, stream>>>(k16, BG, N, d, part);
+    const unsigned blocks = (unsigned)((long long)BG * T);
+    if (d == 128) {
+      if (fp16) kmean_partial_kernel<128, true><<<blocks, 128, 0, stream>>>(k16, N, part);
+      else kmean_partial_kernel<128, false><<<blocks, 128, 0, stream>>>(k16, N, part);
+    } else {
+      if (fp16) kmean_partial_kernel<64, true><<<blocks, 64, 0, stream>>>(k16, N, part);
+      else kmean_partial_kernel<64, false><<<blocks, 64, 0, stream>>>(k16, N, part);
+    }
     TATTN_CUDA(cudaGetLastError());
   }
   kmean_final_kernel<<<(BG * d + 127) / 128, 128, 0, stream>>>(part, BG, N, d, kmean);
@@ -204,14 +216,14 @@ int launch_prepass(const void* q, const void* k, int B, int Hq, int Hkv, int N, 
   const unsigned qblocks = (unsigned)((long long)B * Hkv * T + (long long)B * Hq * T);
   if (d == 128) {
     if (fp16)
-      quant_kernel<128, true><<<qblocks, 256, 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+      quant_kernel<128, true><<<qblocks, quant_threads<128>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
     else
-      quant_kernel<128, false><<<qblocks, 256, 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+      quant_kernel<128, false><<<qblocks, quant_threads<128>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
   } else {
     if (fp16)
-      quant_kernel<64, true><<<qblocks, 256, 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+      quant_kernel<64, true><<<qblocks, quant_threads<64>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
     else
-      quant_kernel<64, false><<<qblocks, 256, 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+      quant_kernel<64, false><<<qblocks, quant_threads<64>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
   }
   TATTN_CUDA(cudaGetLastError());
   return ATTN_OK;

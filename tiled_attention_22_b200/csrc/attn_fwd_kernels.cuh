@@ -75,8 +75,21 @@ struct FwdCfg {
 #define TATTN_POLY_INT8 0
 #endif
   static constexpr int POLY_PER_16 = INT8 ? TATTN_POLY_INT8 : TATTN_POLY_BF16;
-  static constexpr int KSTAGES = (D == 128 && !INT8) ? 2 : 4;
-  static constexpr int VSTAGES = (D == 128) ? (INT8 ? 3 : 2) : 4;
+  // pipeline depth (K and V rings); defaults chosen by measurement on the named workloads
+#ifndef TATTN_KS_128B
+#define TATTN_KS_128B 2
+#endif
+#ifndef TATTN_VS_128B
+#define TATTN_VS_128B 2
+#endif
+#ifndef TATTN_KS_128I
+#define TATTN_KS_128I 4
+#endif
+#ifndef TATTN_VS_128I
+#define TATTN_VS_128I 3
+#endif
+  static constexpr int KSTAGES = D == 128 ? (INT8 ? TATTN_KS_128I : TATTN_KS_128B) : 4;
+  static constexpr int VSTAGES = D == 128 ? (INT8 ? TATTN_VS_128I : TATTN_VS_128B) : 4;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QT * Q_TILE;
   static constexpr int OFF_V = OFF_K + KSTAGES * K_TILE;
@@ -93,12 +106,37 @@ struct FwdCfg {
   static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 };
 
-// 12 warps: two softmax warpgroups and one producer warpgroup (TMA warp, MMA warp, 2 idle).
-constexpr int kFwdThreads = 384;
-constexpr int kLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
-constexpr int kRegsSoftmax = 208;  // per thread, softmax warpgroups
-constexpr int kRegsProducer = 88;  // per thread, producer warpgroup
-static_assert(128 * (2 * kRegsSoftmax + kRegsProducer) <= kFwdThreads * kLaunchRegs, "register split");
+#ifndef TATTN_PFULL_PER_WARP
+#define TATTN_PFULL_PER_WARP 1
+#endif
+
+// Warp roles.  Softmax warps come first, then one producer warpgroup (TMA warp, MMA warp, 2 idle).
+//   SPLIT = false: 8 softmax warps, one thread per score row (32x32b TMEM accesses).
+//   SPLIT = true : 16 softmax warps, four threads per score row (16x256b TMEM accesses): warps w
+//                  and w+4 share a 32-lane TMEM quarter, 16 lanes each, and a row's max is
+//                  reduced over its four threads with warp shuffles.  Each warp does half the
+//                  exp2 work per tile, so a tile's softmax fits in the other tile's MMA time.
+// setmaxnreg moves registers from the producer warpgroup to the softmax warpgroups; the split
+// must fit the registers the CTA is launched with (65536 / threads, rounded down to 8).
+template <bool SPLIT>
+struct FwdRoles {
+  static constexpr int kSoftmaxWarps = SPLIT ? 16 : 8;
+  static constexpr int kThreads = (kSoftmaxWarps + 4) * 32;
+  static constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;
+#ifndef TATTN_SPLIT_REGS_SOFTMAX
+#define TATTN_SPLIT_REGS_SOFTMAX 104
+#endif
+#ifndef TATTN_SPLIT_REGS_PRODUCER
+#define TATTN_SPLIT_REGS_PRODUCER 64
+#endif
+  static constexpr int kRegsSoftmax = SPLIT ? TATTN_SPLIT_REGS_SOFTMAX : 208;
+  static constexpr int kRegsProducer = SPLIT ? TATTN_SPLIT_REGS_PRODUCER : 88;
+  static constexpr int kTmaWarp = kSoftmaxWarps;
+  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr int kThreadsPerTile = kSoftmaxWarps * 16;  // softmax threads per query tile
+  static_assert(128 * (kSoftmaxWarps / 4 * kRegsSoftmax + kRegsProducer) <= kThreads * kLaunchRegs,
+                "register split exceeds the launch registers");
+};
 
 // Wait-site ids recorded with a timeout (role * 16 + barrier kind).
 enum : int { W_LOAD = 0x10, W_MMA = 0x20, W_SOFTMAX = 0x30, W_DRAIN = 0x40, W_PROBE = 0x50 };
@@ -259,12 +297,10 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
   }
   l_run += (ls0.x + ls0.y) + (ls1.x + ls1.y);
   if (rescale && j > 0) {
-    // O holds the P V sums of tiles 0..j-1; the last of them must have landed before the rescale,
-    // and P V of tile j is issued only after this thread arrives on p_full.
-    bool ok = mbar_wait(o_done_t, (j - 1) & 1, abort_flag, W_SOFTMAX + 2);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) return false;
-    tc_fence_after();
+    // O holds the P V sums of key tiles 0..j-1.  The s_full commit that woke this thread was made
+    // after S(j), i.e. after P V(j-1) was issued by the same thread, and a commit tracks every
+    // earlier tcgen05 operation of its thread: P V(j-1) has completed.  P V(j) is issued only
+    // after this thread arrives on p_full.
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
@@ -278,11 +314,118 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
   return true;
 }
 
-template <int D, bool INT8, bool FP16>
-__global__ void __launch_bounds__(kFwdThreads, 1)
+// Split-row variant of softmax_step: this thread holds rows A (lane base + t/4) and B (+8), and
+// of each row the columns 8k + 2(t%4) + {0,1}, k = 0..15 (a 16x256b TMEM load).  Row maxima are
+// reduced over the 4 threads of a row with two xor-shuffles; each thread keeps a partial row sum
+// (summed over the 4 threads in the epilogue).  P goes back with a 16x128b store, which puts the
+// packed pair of columns (8k + 2(t%4), +1) at packed column 4k + t%4 of the same rows.
+template <int D, bool INT8, bool FP16, bool MASKED>
+__device__ __forceinline__ bool softmax_step_split(uint32_t tS, uint32_t tO, float sc, int limA, int limB, int j,
+                                                   float (&m_run)[2], float (&l_run)[2], uint64_t* o_done_t,
+                                                   volatile int* abort_flag) {
+  const int q4 = threadIdx.x & 3;
+  uint32_t r[64];
+  tmem_ld_16x256_x16(tS, r);
+  tmem_ld_wait64(r);
+  float x[64];
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    x[i] = INT8 ? __uint_as_float(r[i] + 0x4B400000u) : __uint_as_float(r[i]);
+    if (MASKED) {
+      const int col = 8 * (i >> 2) + 2 * q4 + (i & 1);
+      if (col >= ((i & 2) ? limB : limA)) x[i] = -INFINITY;
+    }
+  }
+  // repetitions 0..15: rep 0 starts the chains, reps (1,2) ... (13,14) in pairs, rep 15 alone
+  float mA0 = x[0], mA1 = x[1], mB0 = x[2], mB1 = x[3];
+#pragma unroll
+  for (int k = 1; k + 1 < 16; k += 2) {
+    mA0 = max3f(mA0, x[4 * k], x[4 * k + 4]);
+    mA1 = max3f(mA1, x[4 * k + 1], x[4 * k + 5]);
+    mB0 = max3f(mB0, x[4 * k + 2], x[4 * k + 6]);
+    mB1 = max3f(mB1, x[4 * k + 3], x[4 * k + 7]);
+  }
+  float mx[2] = {max3f(mA0, mA1, x[60]), max3f(mB0, mB1, x[62])};
+  mx[0] = fmaxf(mx[0], x[61]);
+  mx[1] = fmaxf(mx[1], x[63]);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+  }
+  float alpha[2] = {1.f, 1.f};
+  bool need_any = false;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float m_tile = INT8 ? (mx[h] - 12582912.0f) * sc : mx[h] * sc;
+    const float m_new = fmaxf(m_run[h], m_tile);
+    if (m_new > m_run[h] + 8.0f) {  // same decision in all 4 threads of the row
+      alpha[h] = ex2_approx(m_run[h] - m_new);
+      l_run[h] *= alpha[h];
+      m_run[h] = m_new;
+      need_any = true;
+    }
+  }
+  const bool rescale = __any_sync(0xffffffffu, need_any);
+  const float2 sc2 = make_float2(sc, sc);
+  const float2 cA = make_float2(-m_run[0], -m_run[0]), cB = make_float2(-m_run[1], -m_run[1]);
+  const float2 off2 = make_float2(-12582912.0f, -12582912.0f);
+  float2 lsA = make_float2(0.f, 0.f), lsB = make_float2(0.f, 0.f);
+  uint32_t pk[32];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float2 xa = make_float2(x[4 * k], x[4 * k + 1]);
+    float2 xb = make_float2(x[4 * k + 2], x[4 * k + 3]);
+    if constexpr (INT8) {
+      xa = fadd2(xa, off2);
+      xb = fadd2(xb, off2);
+    }
+    const float2 a = ffma2(xa, sc2, cA);
+    const float2 b = ffma2(xb, sc2, cB);
+    float pa0, pa1, pb0, pb1;
+    if (!MASKED && (k & 7) >= 8 - FwdCfg<D, INT8>::POLY_PER_16 / 2) {
+      pa0 = exp2_poly(a.x);
+      pa1 = exp2_poly(a.y);
+      pb0 = exp2_poly(b.x);
+      pb1 = exp2_poly(b.y);
+    } else {
+      pa0 = ex2_approx(a.x);
+      pa1 = ex2_approx(a.y);
+      pb0 = ex2_approx(b.x);
+      pb1 = ex2_approx(b.y);
+    }
+    lsA = fadd2(lsA, make_float2(pa0, pa1));
+    lsB = fadd2(lsB, make_float2(pb0, pb1));
+    pk[2 * k] = pack2(pa0, pa1, FP16);
+    pk[2 * k + 1] = pack2(pb0, pb1, FP16);
+  }
+  tmem_st_16x128_x16(tS, pk);
+  l_run[0] += lsA.x + lsA.y;
+  l_run[1] += lsB.x + lsB.y;
+  if (rescale && j > 0) {
+    // O holds the P V sums of key tiles 0..j-1.  The s_full commit that woke this thread was made
+    // after S(j), i.e. after P V(j-1) was issued by the same thread, and a commit tracks every
+    // earlier tcgen05 operation of its thread: P V(j-1) has completed.  P V(j) is issued only
+    // after this thread arrives on p_full.
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      uint32_t o[32];
+      tmem_ld_16x256_x8(tO + 64 * c, o);
+      tmem_ld_wait(o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha[(i >> 1) & 1]);
+      tmem_st_16x256_x8(tO + 64 * c, o);
+    }
+  }
+  return true;
+}
+
+template <int D, bool INT8, bool FP16, bool SPLIT>
+__global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, INT8>;
+  using R = FwdRoles<SPLIT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -304,7 +447,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], TATTN_PFULL_PER_WARP ? R::kThreadsPerTile / 32 : R::kThreadsPerTile);
       mbar_init(&o_done[i], 1);
     }
     for (int i = 0; i < C::KSTAGES; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
@@ -313,11 +456,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == R::kMmaWarp) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == R::kTmaWarp && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -347,21 +490,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int h = (kvz - b * p.Hkv) * G + within % G;
   const int bh = b * p.Hq + h;
   const int nkv = (p.N + 127) / 128;
-  int n_t[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
+  // key tiles each query tile visits (0 for a tile past N); n1 >= n0 unless tile 1 is empty
+  auto key_tiles = [&](int t) {
     const int row0 = mb * 256 + 128 * t;
-    n_t[t] = row0 < p.N ? (p.causal ? min(nkv, row0 / 128 + 1) : nkv) : 0;
-  }
-  const int nmax = max(n_t[0], n_t[1]);
+    return row0 < p.N ? (p.causal ? min(nkv, row0 / 128 + 1) : nkv) : 0;
+  };
+  const int n0 = key_tiles(0), n1 = key_tiles(1);
+  // (kept in registers: a runtime-indexed array would live in local memory)
+  auto n_of = [&](int t) { return t ? n1 : n0; };
+  const int nmax = max(n0, n1);
 
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
 
-  if (warp >= 8) {
-    regs_decrease<kRegsProducer>();
-  if (warp == 8) {
+  if (warp >= R::kSoftmaxWarps) {
+    regs_decrease<R::kRegsProducer>();
+  if (warp == R::kTmaWarp) {
     // ================================ TMA producer ================================
     if (lane == 0) {
       const uint64_t pol_stream = policy_evict_first();
@@ -369,7 +514,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int t = 0; t < 2; ++t) {
-        if (n_t[t] == 0) continue;
+        if (n_of(t) == 0) continue;
         mbar_arrive_expect_tx(&q_full[t], C::Q_TILE);
         for (int pn = 0; pn < C::QK_PANELS; ++pn)
           tma_load_3d(sQ + t * C::Q_TILE + pn * C::QK_PANEL_BYTES, &tmQ, pn * C::QK_BOX_X, mb * 256 + 128 * t, bh,
@@ -393,7 +538,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (!ok) {
         // Drain: every issued copy must land before the CTA's shared memory is released.
         for (int t = 0; t < 2; ++t)
-          if (n_t[t]) mbar_wait(&q_full[t], 0, nullptr, W_DRAIN + 1, 200000000ull);
+          if (n_of(t)) mbar_wait(&q_full[t], 0, nullptr, W_DRAIN + 1, 200000000ull);
         for (int j = max(0, k_issued - C::KSTAGES); j < k_issued; ++j)
           mbar_wait(&k_full[j % C::KSTAGES], (j / C::KSTAGES) & 1, nullptr, W_DRAIN + 2, 200000000ull);
         for (int j = max(0, v_issued - C::VSTAGES); j < v_issued; ++j)
@@ -401,18 +546,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == R::kMmaWarp) {
     // ================================ MMA issuer ================================
     if (lane == 0) {
-      bool ok = true;
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      auto users_first = [&](int j) { return j < n_t[0] ? 0 : 1; };
-      auto users_last = [&](int j) { return j < n_t[1] ? 1 : 0; };
+      bool ok = true;
+      auto users_first = [&](int j) { return j < n0 ? 0 : 1; };
+      auto users_last = [&](int j) { return j < n1 ? 1 : 0; };
       // prologue: S_t(0) for both tiles
       if (nmax > 0) {
         ok = mbar_wait(&k_full[0], 0, abort_flag, W_MMA + 1);
         for (int t = 0; t < 2 && ok; ++t) {
-          if (n_t[t] == 0) continue;
+          if (n_of(t) == 0) continue;
           if (!(ok = mbar_wait(&q_full[t], 0, abort_flag, W_MMA + 2))) break;
           tc_fence_after();
           issue_qk<D, INT8, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr);
@@ -424,7 +569,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int vs = j % C::VSTAGES;
         const int ks1 = (j + 1) % C::KSTAGES;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= n_t[t]) continue;
+          if (j >= n_of(t)) continue;
           if (!(ok = mbar_wait(&p_full[t], j & 1, abort_flag, W_MMA + 3))) break;
           tc_fence_after();
           if (users_first(j) == t) {
@@ -432,9 +577,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tc_fence_after();
           }
           issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
-          mma_commit(&o_done[t]);
+          if (j + 1 == n_of(t)) mma_commit(&o_done[t]);  // the tile's last P V: O is final
           if (users_last(j) == t) mma_commit(&v_empty[vs]);
-          if (j + 1 < n_t[t]) {
+          if (j + 1 < n_of(t)) {
             if (users_first(j + 1) == t) {
               if (!(ok = mbar_wait(&k_full[ks1], ((j + 1) / C::KSTAGES) & 1, abort_flag, W_MMA + 5))) break;
               tc_fence_after();
@@ -452,81 +597,183 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     __syncwarp();
-  }  // warps 10-11: nothing to do
+  }  // remaining producer warps: nothing to do
   } else {
-    regs_increase<kRegsSoftmax>();
-    // ================================ softmax (one row per thread) ================================
-    const int t = warp >> 2, wq = warp & 3;
-    const int nt = n_t[t];
-    const int row0 = mb * 256 + 128 * t;
-    const int row = row0 + wq * 32 + lane;
-    const uint32_t tS = tmem + C::tm_s(t) + ((uint32_t)(wq * 32) << 16);
-    const uint32_t tO = tmem + C::tm_o(t) + ((uint32_t)(wq * 32) << 16);
-    const int nblk = (p.N + 127) / 128;
-    // (an empty tile, row0 >= N, reads nothing: its sq entry does not exist)
-    const float sq_scale = (INT8 && nt > 0) ? p.sq[(size_t)bh * nblk + row0 / 128] * p.scale_log2 : p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      ok = mbar_wait(&s_full[t], j & 1, abort_flag, W_SOFTMAX + 1);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nblk + j]) : sq_scale;
-      if constexpr (INT8) sc = fmaxf(sc, 1e-30f);  // a zero block: keep -inf * sc = -inf for masks
-      // causal diagonal tile (key > query) and the ragged last key tile (key >= N) are masked;
-      // keys [0, lim) of the tile are visible
-      const int col0 = j * 128;
-      const bool diag = p.causal && (j == nt - 1);
-      if (diag || (col0 + 128 > p.N)) {
-        const int lim = (diag ? min(row + 1, p.N) : p.N) - col0;
-        ok = softmax_step<D, INT8, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
-      } else {
-        ok = softmax_step<D, INT8, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
-      }
-      if (!ok) break;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-    }
-    if (ok && nt > 0) {
-      ok = mbar_wait(&o_done[t], (nt - 1) & 1, abort_flag, W_SOFTMAX + 3);
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok) {
+    regs_increase<R::kRegsSoftmax>();
+    if constexpr (SPLIT) {
+      // ============================ softmax, four threads per row ============================
+      const int t = warp >> 3;                  // query tile
+      const int wq = warp & 3;                  // TMEM lane quarter
+      const int half = (warp >> 2) & 1;         // which 16 lanes of the quarter
+      const int lane_base = wq * 32 + half * 16;
+      const int nt = n_of(t);
+      const int row0 = mb * 256 + 128 * t;
+      const int rowA = row0 + lane_base + (lane >> 2), rowB = rowA + 8;
+      const uint32_t tS = tmem + C::tm_s(t) + ((uint32_t)lane_base << 16);
+      const uint32_t tO = tmem + C::tm_o(t) + ((uint32_t)lane_base << 16);
+      const int nblk = (p.N + 127) / 128;
+      const float sq_scale =
+          (INT8 && nt > 0) ? p.sq[(size_t)bh * nblk + row0 / 128] * p.scale_log2 : p.scale_log2;
+      float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+      bool ok = true;
+      for (int j = 0; j < nt; ++j) {
+        ok = mbar_wait(&s_full[t], j & 1, abort_flag, W_SOFTMAX + 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
         tc_fence_after();
-        const float inv_l = 1.0f / l_run;
-        uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)bh * p.N + (size_t)row) * (D * 2);
+        float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nblk + j]) : sq_scale;
+        if constexpr (INT8) sc = fmaxf(sc, 1e-30f);
+        const int col0 = j * 128;
+        const bool diag = p.causal && (j == nt - 1);
+        if (diag || (col0 + 128 > p.N)) {
+          const int limA = (diag ? min(rowA + 1, p.N) : p.N) - col0;
+          const int limB = (diag ? min(rowB + 1, p.N) : p.N) - col0;
+          ok = softmax_step_split<D, INT8, FP16, true>(tS, tO, sc, limA, limB, j, m_run, l_run, &o_done[t],
+                                                       abort_flag);
+        } else {
+          ok = softmax_step_split<D, INT8, FP16, false>(tS, tO, sc, 128, 128, j, m_run, l_run, &o_done[t],
+                                                        abort_flag);
+        }
+        if (!ok) break;
+        tmem_st_wait();
+        tc_fence_before();
+        if (TATTN_PFULL_PER_WARP) {
+          // one arrival per warp: every lane's TMEM stores are complete (wait::st) and fenced
+          // before the warp synchronises; lane 0 then releases them to the MMA thread
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[t]);
+        } else {
+          mbar_arrive(&p_full[t]);
+        }
+      }
+      if (ok && nt > 0) {
+        ok = mbar_wait(&o_done[t], 0, abort_flag, W_SOFTMAX + 3);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          // full row sums: add the partials of the row's four threads
+          float inv_l[2];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_ld_wait(o);
-          uint32_t pk[16];
+          for (int h = 0; h < 2; ++h) {
+            l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
+            l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
+            inv_l[h] = 1.0f / l_run[h];
+          }
+          const int q4 = lane & 3;
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, FP16);
-          if (row < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t o[32];
+            tmem_ld_16x256_x8(tO + 64 * c, o);
+            tmem_ld_wait(o);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int k = 0; k < 8; ++k) {
+              const int col = 64 * c + 8 * k + 2 * q4;
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int row = h ? rowB : rowA;
+                const uint32_t v = pack2(__uint_as_float(o[4 * k + 2 * h]) * inv_l[h],
+                                         __uint_as_float(o[4 * k + 2 * h + 1]) * inv_l[h], FP16);
+                if (row < p.N)
+                  *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.o) +
+                                               (((size_t)bh * p.N + row) * D + col) * 2) = v;
+              }
+            }
+          }
+          if (p.lse != nullptr && q4 == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int row = h ? rowB : rowA;
+              if (row < p.N) {
+                float lse = (m_run[h] + __log2f(l_run[h])) * 0.69314718055994531f;
+                if constexpr (INT8) lse += p.bias[(size_t)bh * p.N + row];
+                p.lse[(size_t)bh * p.N + row] = lse;
+              }
+            }
           }
         }
-        if (p.lse != nullptr && row < p.N) {
-          float lse = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-          if constexpr (INT8) lse += p.bias[(size_t)bh * p.N + row];
-          p.lse[(size_t)bh * p.N + row] = lse;
+      }
+      if (!ok) tmem_st_wait();
+    } else {
+      // ================================ softmax (one row per thread) ================================
+      const int t = warp >> 2, wq = warp & 3;
+      const int nt = n_of(t);
+      const int row0 = mb * 256 + 128 * t;
+      const int row = row0 + wq * 32 + lane;
+      const uint32_t tS = tmem + C::tm_s(t) + ((uint32_t)(wq * 32) << 16);
+      const uint32_t tO = tmem + C::tm_o(t) + ((uint32_t)(wq * 32) << 16);
+      const int nblk = (p.N + 127) / 128;
+      // (an empty tile, row0 >= N, reads nothing: its sq entry does not exist)
+      const float sq_scale = (INT8 && nt > 0) ? p.sq[(size_t)bh * nblk + row0 / 128] * p.scale_log2 : p.scale_log2;
+      float m_run = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nt; ++j) {
+        ok = mbar_wait(&s_full[t], j & 1, abort_flag, W_SOFTMAX + 1);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nblk + j]) : sq_scale;
+        if constexpr (INT8) sc = fmaxf(sc, 1e-30f);  // a zero block: keep -inf * sc = -inf for masks
+        // causal diagonal tile (key > query) and the ragged last key tile (key >= N) are masked;
+        // keys [0, lim) of the tile are visible
+        const int col0 = j * 128;
+        const bool diag = p.causal && (j == nt - 1);
+        if (diag || (col0 + 128 > p.N)) {
+          const int lim = (diag ? min(row + 1, p.N) : p.N) - col0;
+          ok = softmax_step<D, INT8, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
+        } else {
+          ok = softmax_step<D, INT8, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
+        }
+        if (!ok) break;
+        tmem_st_wait();
+        tc_fence_before();
+        if (TATTN_PFULL_PER_WARP) {
+          // one arrival per warp: every lane's TMEM stores are complete (wait::st) and fenced
+          // before the warp synchronises; lane 0 then releases them to the MMA thread
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[t]);
+        } else {
+          mbar_arrive(&p_full[t]);
         }
       }
-    }
-    if (!ok) {
-      // make sure this thread's TMEM traffic is finished before teardown
-      tmem_st_wait();
+      if (ok && nt > 0) {
+        ok = mbar_wait(&o_done[t], 0, abort_flag, W_SOFTMAX + 3);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          const float inv_l = 1.0f / l_run;
+          uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)bh * p.N + (size_t)row) * (D * 2);
+  #pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_ld_wait(o);
+            uint32_t pk[16];
+  #pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, FP16);
+            if (row < p.N) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+  #pragma unroll
+              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+          if (p.lse != nullptr && row < p.N) {
+            float lse = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+            if constexpr (INT8) lse += p.bias[(size_t)bh * p.N + row];
+            p.lse[(size_t)bh * p.N + row] = lse;
+          }
+        }
+      }
+      if (!ok) {
+        // make sure this thread's TMEM traffic is finished before teardown
+        tmem_st_wait();
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == R::kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

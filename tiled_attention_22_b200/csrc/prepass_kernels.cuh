@@ -9,7 +9,8 @@
 // amax/127, code = clamp(rint(x * (127/amax)), -127, 127) with ties to even; a zero block gets scale 0.
 //
 // These kernels are HBM-bound: plain 16-byte vector loads and stores, no tensor cores.
-//   kmean_partial_kernel  K -> float64 partial sums per 128-token block (sequential in token order)
+//   kmean_partial_kernel  K -> float64 partial sums per 128-token block (sequential in token order,
+//                         the block staged in shared memory)
 //   kmean_final_kernel    partials -> mean (sequential in block order), (float)(total / N)
 //   quant_kernel          K blocks: smooth + quantise -> k8, sk;  Q blocks: quantise -> q8, sq and
 //                         the lse bias scale * q_i . mean (row dot product, warp-shuffle reduced)
@@ -20,6 +21,13 @@
 #include <cstdint>
 
 namespace tattn {
+
+// max(a, |b|, |c|) in one instruction
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+  return d;
+}
 
 template <bool FP16>
 __device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
@@ -40,47 +48,35 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
   }
 }
 
-// One thread = one (batch*kv head, 128-token block, 8-channel chunk).  Adds the block's tokens in
-// ascending order into float64 accumulators (one per channel), starting from 0.0.
-template <bool FP16>
-__global__ void __launch_bounds__(128) kmean_partial_kernel(const uint16_t* __restrict__ k, int BG, int N, int d,
-                                                             double* __restrict__ part) {
-  const int chunks = d / 8;
+// One CTA (D threads) per (batch*kv head, 128-token block): the block is staged in shared memory
+// with 16-byte loads (whole rows, so each DRAM page is read in one sweep), then thread c adds
+// channel c's tokens in ascending order into a float64 partial starting at 0.0.
+template <int D, bool FP16>
+__global__ void __launch_bounds__(D) kmean_partial_kernel(const uint16_t* __restrict__ k, int N,
+                                                           double* __restrict__ part) {
+  __shared__ __align__(16) uint16_t tile[128 * D];
   const int T = (N + 127) / 128;
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)BG * T * chunks) return;
-  const int chunk = (int)(idx % chunks);
-  const long long rest = idx / chunks;
-  const int t = (int)(rest % T);
-  const int bg = (int)(rest / T);
+  const int t = blockIdx.x % T;
+  const int bg = blockIdx.x / T;
   const int cnt = min(128, N - t * 128);
-  const uint4* src = reinterpret_cast<const uint4*>(k + ((size_t)bg * N + (size_t)t * 128) * d + chunk * 8);
-  const int stride = d / 8;  // uint4 per row
-  double acc[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = 0.0;
-  int i = 0;
-  for (; i + 8 <= cnt; i += 8) {
-    uint4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = __ldg(src + (size_t)(i + u) * stride);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      float x[8];
-      unpack8<FP16>(v[u], x);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = __dadd_rn(acc[c], (double)x[c]);
-    }
+  const uint4* src = reinterpret_cast<const uint4*>(k + ((size_t)bg * N + (size_t)t * 128) * D);
+  uint4* dst = reinterpret_cast<uint4*>(tile);
+  const int n16 = cnt * D / 8;  // 16-byte chunks in the block
+#pragma unroll 4
+  for (int i = threadIdx.x; i < n16; i += D) dst[i] = __ldg(src + i);
+  __syncthreads();
+  const int c = threadIdx.x;
+  double acc = 0.0;
+  for (int i = 0; i < cnt; ++i) {
+    const uint16_t b = tile[i * D + c];
+    float x;
+    if constexpr (FP16)
+      x = __half2float(__ushort_as_half(b));
+    else
+      x = __uint_as_float((uint32_t)b << 16);
+    acc = __dadd_rn(acc, (double)x);
   }
-  for (; i < cnt; ++i) {
-    float x[8];
-    unpack8<FP16>(__ldg(src + (size_t)i * stride), x);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = __dadd_rn(acc[c], (double)x[c]);
-  }
-  double* dst = part + ((size_t)bg * T + t) * d + chunk * 8;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) dst[c] = acc[c];
+  part[((size_t)bg * T + t) * D + c] = acc;
 }
 
 // One thread = one (batch*kv head, channel): total over blocks in ascending order, then the mean.
@@ -96,19 +92,27 @@ __global__ void __launch_bounds__(128) kmean_final_kernel(const double* __restri
   kmean[idx] = __double2float_rn(__ddiv_rn(total, (double)N));
 }
 
-// 256 threads per CTA, one CTA per 128-token block.  Blocks [0, nK) are K blocks (b, g, t),
-// blocks [nK, nK + nQ) are Q blocks (b, h, t).  Thread layout: d/16 threads per row, each holding
-// 16 consecutive channels; rows are covered in passes of 256 / (d/16) rows.
+// One CTA per 128-token block (4*D threads: 512 for d=128, 256 for d=64).  Blocks [0, nK) are K
+// blocks (b, g, t), blocks [nK, nK + nQ) are Q blocks (b, h, t).  Thread layout: d/8 threads per
+// row, each holding 8 consecutive channels (one 16-byte load per row); rows are covered in
+// 4 passes of 32 rows.  The block stays in registers as raw 16-bit pairs; it is unpacked once for
+// the absmax (and Q's bias dot product) and again for quantisation, which keeps the register
+// count at 64 (1024 resident threads per SM, 64 KB of loads in flight).
+template <int D>
+constexpr int quant_threads() { return 4 * D; }
+
 template <int D, bool FP16>
-__global__ void __launch_bounds__(256) quant_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
-                                                     int B, int Hq, int Hkv, int N, float scale,
-                                                     const float* __restrict__ kmean, int8_t* __restrict__ q8,
-                                                     float* __restrict__ sq, int8_t* __restrict__ k8,
-                                                     float* __restrict__ sk, float* __restrict__ bias) {
-  constexpr int TPR = D / 16;           // threads per row
-  constexpr int RPP = 256 / TPR;        // rows per pass
-  constexpr int PASSES = 128 / RPP;
-  __shared__ float warp_max[8];
+__global__ void __launch_bounds__(4 * D, 256 / D) quant_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                                                        int B, int Hq, int Hkv, int N, float scale,
+                                                        const float* __restrict__ kmean, int8_t* __restrict__ q8,
+                                                        float* __restrict__ sq, int8_t* __restrict__ k8,
+                                                        float* __restrict__ sk, float* __restrict__ bias) {
+  constexpr int NT = 4 * D;
+  constexpr int TPR = D / 8;            // threads per row
+  constexpr int RPP = NT / TPR;         // rows per pass (32)
+  constexpr int PASSES = 128 / RPP;     // 4
+  constexpr int NW = NT / 32;
+  __shared__ float warp_max[NW];
 
   const int T = (N + 127) / 128;
   const int nK = B * Hkv * T;
@@ -123,89 +127,75 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint16_t* __restrict__
   const int tid = threadIdx.x;
   const int chunk = tid % TPR, r_in = tid / TPR;
 
-  float mean[16];
+  float mean[8];
   {
-    const float4* m4 = reinterpret_cast<const float4*>(kmean + (size_t)g_mean * D + chunk * 16);
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const float4 m = __ldg(m4 + v);
-      mean[4 * v] = m.x;
-      mean[4 * v + 1] = m.y;
-      mean[4 * v + 2] = m.z;
-      mean[4 * v + 3] = m.w;
-    }
+    const float4* m4 = reinterpret_cast<const float4*>(kmean + (size_t)g_mean * D + chunk * 8);
+    const float4 a = __ldg(m4), b = __ldg(m4 + 1);
+    mean[0] = a.x; mean[1] = a.y; mean[2] = a.z; mean[3] = a.w;
+    mean[4] = b.x; mean[5] = b.y; mean[6] = b.z; mean[7] = b.w;
   }
 
-  float x[PASSES][16];
+  float x[PASSES][8];
+  {
+    uint4 raw[PASSES];
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int row = ps * RPP + r_in;
+      raw[ps] = row < cnt ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)row * D + chunk * 8))
+                          : make_uint4(0, 0, 0, 0);  // +0.0 in both 16-bit formats
+    }
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) unpack8<FP16>(raw[ps], x[ps]);
+  }
   float amax = 0.f;
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
     const int row = ps * RPP + r_in;
     const bool valid = row < cnt;  // uniform over the TPR lanes of one row
-    if (valid) {
-      const uint4* s4 = reinterpret_cast<const uint4*>(src + (size_t)row * D + chunk * 16);
-      float lo[8], hi[8];
-      unpack8<FP16>(__ldg(s4), lo);
-      unpack8<FP16>(__ldg(s4 + 1), hi);
+    if (is_k) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        x[ps][c] = lo[c];
-        x[ps][8 + c] = hi[c];
-      }
-      if (is_k) {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) x[ps][c] = __fsub_rn(x[ps][c], mean[c]);
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 16; ++c) x[ps][c] = 0.f;
-    }
-    if (!is_k) {  // CTA-uniform branch
-      // lse bias: scale * q_row . mean; 16 channels per lane, then a shuffle sum over the row's lanes
+      for (int c = 0; c < 8; ++c) x[ps][c] = valid ? __fsub_rn(x[ps][c], mean[c]) : 0.f;
+    } else {  // CTA-uniform branch
+      // lse bias: scale * q_row . mean; 8 channels per lane, then a shuffle sum over the row's lanes
       float dot = 0.f;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) dot = fmaf(x[ps][c], mean[c], dot);
+      for (int c = 0; c < 8; ++c) dot = fmaf(x[ps][c], mean[c], dot);
 #pragma unroll
       for (int off = TPR / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
       if (valid && chunk == 0) bias[(size_t)bh * N + (size_t)t * 128 + row] = scale * dot;
     }
 #pragma unroll
-    for (int c = 0; c < 16; ++c) amax = fmaxf(amax, fabsf(x[ps][c]));
+    for (int c = 0; c < 8; c += 2) amax = max3_abs(amax, x[ps][c], x[ps][c + 1]);
   }
-  // block absmax: warp shuffle, then across the 8 warps
+  // block absmax: warp shuffle, then across the warps
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   if ((tid & 31) == 0) warp_max[tid >> 5] = amax;
   __syncthreads();
   amax = warp_max[0];
 #pragma unroll
-  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
+  for (int w = 1; w < NW; ++w) amax = fmaxf(amax, warp_max[w]);
 
   const bool zero = (amax == 0.f);
   const float scl = zero ? 0.f : __fdiv_rn(amax, 127.0f);
   const float inv = zero ? 0.f : __fdiv_rn(127.0f, amax);
   if (tid == 0) (is_k ? sk : sq)[(size_t)bh * T + t] = scl;
 
+  // code = rint(fl(x * inv)): the product is rounded once (__fmul_rn), then adding 1.5 * 2^23
+  // rounds it to the nearest integer, ties to even (float32 spacing is 1 on [2^23, 2^24)), and the
+  // low byte of the sum's bit pattern is the code in two's complement.  No clamp is needed:
+  // |x| <= amax and inv <= (127/amax)(1 + 2^-24), so |fl(x * inv)| < 127.5 and |code| <= 127.
+  // (A zero block has inv = 0 and gives code 0.)
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
     const int row = ps * RPP + r_in;
     if (row < cnt) {
-      uint32_t w[4];
+      uint32_t b[8];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint32_t packed = 0;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          int code = 0;
-          if (!zero) {
-            code = __float2int_rn(__fmul_rn(x[ps][4 * v + c], inv));
-            code = max(-127, min(127, code));
-          }
-          packed |= (uint32_t)(code & 0xff) << (8 * c);
-        }
-        w[v] = packed;
-      }
-      *reinterpret_cast<uint4*>(dst + (size_t)row * D + chunk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int c = 0; c < 8; ++c) b[c] = __float_as_uint(__fadd_rn(__fmul_rn(x[ps][c], inv), 12582912.0f));
+      const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+      const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+      *reinterpret_cast<uint2*>(dst + (size_t)row * D + chunk * 8) = make_uint2(w0, w1);
     }
   }
 }
