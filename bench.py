@@ -37,6 +37,38 @@ sys.path.insert(0, ROOT)
 from attn_workloads import WORKLOADS, make_inputs  # noqa: E402
 
 
+KERNEL_SOURCES = ("tiled_attention_22_b200/csrc/attn_fwd_kernels.cuh", "tiled_attention_22_b200/csrc/ptx.cuh",
+                  "tiled_attention_22_b200/csrc/api.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_kernel_traffic_mha_causal_b4_h32_n4096_d128.txt")
+
+
+def _kernel_source_hash():
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _measured_traffic(mode):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary, or None when the
+    kernel sources changed since those counters were taken (or no summary exists)."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    fields = {}
+    with open(TRAFFIC_FILE) as f:
+        for line in f:
+            if "=" in line and not line.lstrip().startswith("#"):
+                key, val = line.split("=", 1)
+                fields[key.strip()] = val.strip()
+    if fields.get("kernel_source_sha256") != _kernel_source_hash():
+        return None
+    val = fields.get(f"{mode}_dram_bytes_per_launch")
+    return int(val) if val else None
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -339,10 +371,13 @@ def run_native(args, w, world, rank, local):
                         "fused_tflops": achieved,
                         "prepass_gbs": _prepass_bytes(w) / (r8["kernel_ms"][0] * 1e-3) / 1e9},
             "bf16_exact": {"tflops": rb["tflops"], "ms_per_step": rb["ms_per_step"],
-                           "frac_of_bf16_peak": (flops / (rb["kernel_ms"][0] * 1e-3) / 1e12) / bf16_peak},
+                           "frac_of_bf16_peak": (flops / (rb["kernel_ms"][0] * 1e-3) / 1e12) / bf16_peak,
+                           "traffic": _measured_traffic("bf16_exact"),
+                           "algorithmic_bytes": _fused_bytes(w, "bf16_exact")},
         },
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": mixed_peak, "unit": "TFLOP/s",
-                     "frac": achieved / mixed_peak, "traffic": None,
+                     "frac": achieved / mixed_peak, "traffic": _measured_traffic("int8_qk"),
+                     "algorithmic_bytes": _fused_bytes(w, "int8_qk"),
                      "kernel": "attn_fwd_kernel<128,int8,bf16>",
                      "peak_note": ("4/3 x measured bf16 %s (%s): INT8 half of the FLOPs at 2x the bf16 rate"
                                    % ("sustained" if long_region else "burst", peaks["source"]))},
@@ -354,6 +389,17 @@ def run_native(args, w, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     return line
+
+
+def _fused_bytes(w, mode):
+    """Algorithmic bytes of one fused-kernel launch: Q and K read once (1 B/elt as INT8 codes,
+    2 B/elt in bf16_exact), V read once, O written once, lse written (4 B/row); scales and the
+    lse bias are per block / per row."""
+    nq = w.B * w.Hq * w.N * w.d
+    nk = w.B * w.Hkv * w.N * w.d
+    qk = 1 if mode == "int8_qk" else 2
+    extra = 4 * w.B * w.Hq * w.N * (2 if mode == "int8_qk" else 1)  # lse (+ bias)
+    return qk * nq + qk * nk + 2 * nk + 2 * nq + extra
 
 
 def _prepass_bytes(w):

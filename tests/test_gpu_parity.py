@@ -288,17 +288,21 @@ def test_canaries_around_outputs(ta, mode):
     assert torch.isfinite(o).all() and torch.isfinite(l).all()
 
 
-def test_host_buffer_entry_point_matches_device_call(ta):
-    w = Workload("t", 1, 4, 2, 500, 128, True, "bf16", "k_offset", 99500)
+@pytest.mark.parametrize("shape", [(1, 4, 2, 500, 128), (3, 6, 3, 333, 64), (2, 8, 8, 1024, 128)])
+def test_host_buffer_entry_point_matches_device_call(ta, shape):
+    """attn_fwd_host pipelines copies and compute over chunks of (batch, kv head) units; its host
+    outputs must equal the device call's bit for bit (odd N exercises 4-unit-aligned chunks)."""
+    B, Hq, Hkv, N, d = shape
+    w = Workload("t", B, Hq, Hkv, N, d, True, "bf16", "k_offset", 99500 + N)
     q, k, v = make_inputs(w)
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     oh = torch.empty_like(qh).pin_memory()
-    lh = torch.empty((1, 4, 500), dtype=torch.float32).pin_memory()
+    lh = torch.empty((B, Hq, N), dtype=torch.float32).pin_memory()
     for mode in ("bf16_exact", "int8_qk"):
         dq, dk, dv = torch.empty_like(q, device="cuda"), torch.empty_like(k, device="cuda"), torch.empty_like(v, device="cuda")
         do = torch.empty_like(dq)
-        dl = torch.empty((1, 4, 500), device="cuda", dtype=torch.float32)
-        ws_bytes = ta.attn_workspace_bytes(1, 4, 2, 500, 128, mode)
+        dl = torch.empty((B, Hq, N), device="cuda", dtype=torch.float32)
+        ws_bytes = ta.attn_workspace_bytes(B, Hq, Hkv, N, d, mode)
         ws = torch.empty(max(ws_bytes, 1), device="cuda", dtype=torch.uint8) if ws_bytes else None
         ta.attn_fwd_host(qh, kh, vh, oh, lh, dq, dk, dv, do, dl, causal=True, mode=mode, workspace=ws)
         o_ref, l_ref = ta.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, mode=mode)

@@ -413,17 +413,92 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   if (!q || !k || !v || !o) return ATTN_ERR_ARG;
   int rc = check_common(dq, dk, dv, do_, dlse, B, Hq, Hkv, N, d, causal, scale, dtype);
   if (rc) return rc;
+  if (mode == ATTN_MODE_INT8_QK && (!workspace || ws_bytes < attn_workspace_bytes(B, Hq, Hkv, N, d, mode)))
+    return ATTN_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t qbytes = (size_t)B * Hq * N * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
-  TATTN_CUDA(cudaMemcpyAsync(dq, q, qbytes, cudaMemcpyHostToDevice, st));
-  TATTN_CUDA(cudaMemcpyAsync(dk, k, kvbytes, cudaMemcpyHostToDevice, st));
-  TATTN_CUDA(cudaMemcpyAsync(dv, v, kvbytes, cudaMemcpyHostToDevice, st));
-  float* dl = (lse && dlse) ? dlse : nullptr;
-  rc = attn_fwd(dq, dk, dv, do_, dl, B, Hq, Hkv, N, d, causal, scale, mode, dtype, workspace, ws_bytes, stream);
-  if (rc) return rc;
-  TATTN_CUDA(cudaMemcpyAsync(o, do_, qbytes, cudaMemcpyDeviceToHost, st));
-  if (dl) TATTN_CUDA(cudaMemcpyAsync(lse, dl, (size_t)B * Hq * N * 4, cudaMemcpyDeviceToHost, st));
-  TATTN_CUDA(cudaStreamSynchronize(st));
+  const bool want_lse = lse && dlse;
+  // Units are (batch, kv head) pairs with their G query heads: independent problems whose Q, K, V,
+  // O and lse slices are contiguous, in unit order, in every [B, H, N, d] tensor.  A run of units
+  // is therefore one contiguous problem with B' = 1, Hq' = n*G, Hkv' = n.  The units are split
+  // into chunks; chunk c's inputs are copied in on a helper stream while chunk c-1 computes on
+  // the caller's stream, and its outputs are copied out on a second helper stream.
+  const int G = Hq / Hkv;
+  const int units = B * Hkv;
+  const int nchunk = units < 8 ? units : 8;
+  const size_t q_unit = (size_t)G * N * d * 2, kv_unit = (size_t)N * d * 2, l_unit = (size_t)G * N * 4;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_in[8] = {}, ev_done[8] = {};
+  auto cleanup = [&]() {
+    for (int c = 0; c < 8; ++c) {
+      if (ev_in[c]) cudaEventDestroy(ev_in[c]);
+      if (ev_done[c]) cudaEventDestroy(ev_done[c]);
+    }
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+  };
+#define TATTN_CUDA_C(call)                          \
+  do {                                              \
+    cudaError_t e_ = (call);                        \
+    if (e_ != cudaSuccess) {                        \
+      cleanup();                                    \
+      return cuda_fail(e_, #call);                  \
+    }                                               \
+  } while (0)
+  TATTN_CUDA_C(cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking));
+  TATTN_CUDA_C(cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking));
+  for (int c = 0; c < nchunk; ++c) {
+    TATTN_CUDA_C(cudaEventCreateWithFlags(&ev_in[c], cudaEventDisableTiming));
+    TATTN_CUDA_C(cudaEventCreateWithFlags(&ev_done[c], cudaEventDisableTiming));
+  }
+  // inputs may still be in use by earlier work on the caller's stream: start after it
+  TATTN_CUDA_C(cudaEventRecord(ev_done[0], st));
+  TATTN_CUDA_C(cudaStreamWaitEvent(s_in, ev_done[0], 0));
+  // lse slices must stay 16-byte aligned: 4 units always are (4 * G * N * 4 bytes)
+  const int align_units = (l_unit % 16 == 0) ? 1 : 4;
+  auto chunk_begin = [&](int c) {
+    if (c >= nchunk) return units;
+    return (int)((long long)units * c / nchunk) / align_units * align_units;
+  };
+  for (int c = 0; c < nchunk; ++c) {
+    const int u0 = chunk_begin(c), n = chunk_begin(c + 1) - u0;
+    if (n <= 0) continue;
+    TATTN_CUDA_C(cudaMemcpyAsync(static_cast<uint8_t*>(dq) + u0 * q_unit, static_cast<const uint8_t*>(q) + u0 * q_unit,
+                                 n * q_unit, cudaMemcpyHostToDevice, s_in));
+    TATTN_CUDA_C(cudaMemcpyAsync(static_cast<uint8_t*>(dk) + u0 * kv_unit,
+                                 static_cast<const uint8_t*>(k) + u0 * kv_unit, n * kv_unit, cudaMemcpyHostToDevice,
+                                 s_in));
+    TATTN_CUDA_C(cudaMemcpyAsync(static_cast<uint8_t*>(dv) + u0 * kv_unit,
+                                 static_cast<const uint8_t*>(v) + u0 * kv_unit, n * kv_unit, cudaMemcpyHostToDevice,
+                                 s_in));
+    TATTN_CUDA_C(cudaEventRecord(ev_in[c], s_in));
+  }
+  for (int c = 0; c < nchunk; ++c) {
+    const int u0 = chunk_begin(c), n = chunk_begin(c + 1) - u0;
+    if (n <= 0) continue;
+    TATTN_CUDA_C(cudaStreamWaitEvent(st, ev_in[c], 0));
+    rc = attn_fwd(static_cast<uint8_t*>(dq) + u0 * q_unit, static_cast<uint8_t*>(dk) + u0 * kv_unit,
+                  static_cast<uint8_t*>(dv) + u0 * kv_unit, static_cast<uint8_t*>(do_) + u0 * q_unit,
+                  want_lse ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(dlse) + u0 * l_unit) : nullptr, 1,
+                  n * G, n, N, d, causal, scale, mode, dtype, workspace, ws_bytes, stream);
+    if (rc) {
+      cudaStreamSynchronize(s_in);
+      cudaStreamSynchronize(st);
+      cleanup();
+      return rc;
+    }
+    TATTN_CUDA_C(cudaEventRecord(ev_done[c], st));
+    TATTN_CUDA_C(cudaStreamWaitEvent(s_out, ev_done[c], 0));
+    TATTN_CUDA_C(cudaMemcpyAsync(static_cast<uint8_t*>(o) + u0 * q_unit, static_cast<uint8_t*>(do_) + u0 * q_unit,
+                                 n * q_unit, cudaMemcpyDeviceToHost, s_out));
+    if (want_lse)
+      TATTN_CUDA_C(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(lse) + u0 * l_unit,
+                                   reinterpret_cast<uint8_t*>(dlse) + u0 * l_unit, n * l_unit, cudaMemcpyDeviceToHost,
+                                   s_out));
+  }
+  TATTN_CUDA_C(cudaStreamSynchronize(s_out));
+  TATTN_CUDA_C(cudaStreamSynchronize(st));
+#undef TATTN_CUDA_C
+  cleanup();
   return ATTN_OK;
 }
 
