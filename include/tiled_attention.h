@@ -198,8 +198,9 @@ int attn_test_wait_timeout(int limit_us, void* stream);
  * attn_test_exp2 - test hook: y[i] = 2^x[i] computed by one of the two exp2 routines the fused
  * kernel's softmax uses: use_poly = 1 -> the FMA-pipe routine (range reduction to [-1/2, 1/2]
  * plus a degree-3 minimax polynomial, relative error <= 7.5e-5 for -125 <= x <= 8; inputs below
- * -125 return 2^-125), use_poly = 0 -> the MUFU ex2.approx instruction.  x, y: device float32
- * arrays of n >= 1 elements.
+ * -125 return 2^-125), use_poly = 2 -> the same routine on packed pairs (f32x2 arithmetic; must
+ * equal use_poly = 1 bit for bit), use_poly = 0 -> the MUFU ex2.approx instruction.  x, y:
+ * device float32 arrays of n >= 1 elements.
  */
 int attn_test_exp2(const float* x, float* y, int n, int use_poly, void* stream);
 

@@ -328,8 +328,10 @@ def test_kernel_exp2_against_cuda_exp2f(ta, use_poly):
     polynomial's bound is its Remez fit (7.5e-5 relative) plus float32 rounding; ex2.approx is
     documented to about 2 ulp."""
     x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, -1e-7, 7.999])]).cuda()
-    y = ta.attn_test_exp2(x, use_poly)
+    y = ta.attn_test_exp2(x, 1 if use_poly else 0)
     ref = torch.exp2(x.double())
     rel = ((y.double() - ref).abs() / ref).max().item()
     assert rel <= (8e-5 if use_poly else 1e-6), rel
     assert torch.isfinite(y).all()
+    if use_poly:
+        assert torch.equal(ta.attn_test_exp2(x, 2), y)  # packed pairs: the same bits

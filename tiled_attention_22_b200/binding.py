@@ -250,9 +250,10 @@ def attn_test_wait_timeout(limit_us: int, stream=None) -> None:
     _check(load_library().attn_test_wait_timeout(int(limit_us), _stream(stream)), "attn_test_wait_timeout")
 
 
-def attn_test_exp2(x, use_poly: bool, stream=None):
-    """Apply the kernel's exp2 routine (polynomial or MUFU) to a float32 CUDA tensor."""
+def attn_test_exp2(x, use_poly, stream=None):
+    """Apply the kernel's exp2 routine to a float32 CUDA tensor: use_poly 0 = MUFU ex2.approx,
+    1 = FMA-pipe polynomial, 2 = the polynomial on packed pairs."""
     y = torch.empty_like(x)
-    _check(load_library().attn_test_exp2(_ptr(x), _ptr(y), x.numel(), int(bool(use_poly)), _stream(stream)),
+    _check(load_library().attn_test_exp2(_ptr(x), _ptr(y), x.numel(), int(use_poly), _stream(stream)),
            "attn_test_exp2")
     return y

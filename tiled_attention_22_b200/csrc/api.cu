@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -21,6 +22,7 @@ namespace {
 using namespace tattn;
 
 thread_local char g_last_cuda_error[256] = "";
+constexpr int kMaxDevices = 64;
 
 int cuda_fail(cudaError_t e, const char* what) {
   std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
@@ -104,17 +106,25 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
   if ((rc = make_map(&tk, k, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hkv, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
   if ((rc = make_map(&tv, v, v_dt, 2, D, p.N, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
   auto kern = attn_fwd_kernel<D, INT8, FP16, SPLIT>;
-  TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-  // The kernel moves registers between warpgroups with setmaxnreg; the increase only completes if
-  // the registers the CTA is launched with cover the split.  Refuse to launch otherwise.
-  cudaFuncAttributes attr;
-  TATTN_CUDA(cudaFuncGetAttributes(&attr, kern));
-  if ((long long)attr.numRegs * R::kThreads <
-          128LL * (R::kSoftmaxWarps / 4 * R::kRegsSoftmax + R::kRegsProducer) ||
-      attr.maxThreadsPerBlock < R::kThreads) {
-    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
-                  "fused kernel built with %d registers/thread: too few for its register split", attr.numRegs);
-    return ATTN_ERR_LAUNCH;
+  // Once per device: allow the dynamic shared memory, and check the register split.  The kernel
+  // moves registers between warpgroups with setmaxnreg; the increase only completes if the
+  // registers the CTA is launched with cover the split, so refuse to launch otherwise.
+  static std::atomic<int> checked[kMaxDevices];
+  int dev = 0;
+  TATTN_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_LAUNCH;
+  if (checked[dev].load(std::memory_order_acquire) != 1) {
+    TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    cudaFuncAttributes attr;
+    TATTN_CUDA(cudaFuncGetAttributes(&attr, kern));
+    if ((long long)attr.numRegs * R::kThreads <
+            128LL * (R::kSoftmaxWarps / 4 * R::kRegsSoftmax + R::kRegsProducer) ||
+        attr.maxThreadsPerBlock < R::kThreads) {
+      std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                    "fused kernel built with %d registers/thread: too few for its register split", attr.numRegs);
+      return ATTN_ERR_LAUNCH;
+    }
+    checked[dev].store(1, std::memory_order_release);
   }
   const long long grid = (long long)p.n_mblocks * p.B * p.Hq;
   kern<<<(unsigned)grid, R::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
@@ -241,6 +251,16 @@ int fwd_int8_quantized(const int8_t* q8, const float* sq, const int8_t* k8, cons
 
 __global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int use_poly) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (use_poly == 2) {  // packed pairs, as the softmax evaluates them
+    if (2 * i + 1 < n) {
+      const float2 r = exp2_poly2(make_float2(x[2 * i], x[2 * i + 1]));
+      y[2 * i] = r.x;
+      y[2 * i + 1] = r.y;
+    } else if (2 * i < n) {
+      y[2 * i] = exp2_poly2(make_float2(x[2 * i], 0.f)).x;
+    }
+    return;
+  }
   if (i < n) y[i] = use_poly ? exp2_poly(x[i]) : ex2_approx(x[i]);
 }
 
@@ -269,7 +289,6 @@ __global__ void wait_forever_probe_kernel(unsigned long long limit_ns) {
 constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB = 1 Mi float64 partials
 static __device__ __align__(256) double g_static_kmean_scratch[kStaticScratchBytes / sizeof(double)];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_static_scratch_mu;
 void* g_static_scratch_addr[kMaxDevices] = {};
 

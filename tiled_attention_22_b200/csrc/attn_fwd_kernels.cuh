@@ -67,14 +67,16 @@ struct FwdCfg {
   static constexpr int V_PANEL_BYTES = BN * 128;
   static constexpr int V_TILE = BN * D * 2;
   static constexpr int PV_STEPS = BN / 16;
-  // of every 16 score columns, how many take exp2_poly (FMA pipe) instead of MUFU ex2
-#ifndef TATTN_POLY_BF16
-#define TATTN_POLY_BF16 0
+  // Of every 16 score columns, how many take exp2_poly (FMA pipe) instead of MUFU ex2.  Measured
+  // on the named workloads: it pays only where the exponentials outweigh the MMA work most
+  // (d = 64: +3% in INT8 mode); at d = 128 every share tried was slower, so it is off there.
+#ifndef TATTN_POLY_D128
+#define TATTN_POLY_D128 0
 #endif
-#ifndef TATTN_POLY_INT8
-#define TATTN_POLY_INT8 0
+#ifndef TATTN_POLY_D64
+#define TATTN_POLY_D64 4
 #endif
-  static constexpr int POLY_PER_16 = INT8 ? TATTN_POLY_INT8 : TATTN_POLY_BF16;
+  static constexpr int POLY_PER_16 = D == 64 ? TATTN_POLY_D64 : TATTN_POLY_D128;
   // pipeline depth (K and V rings); defaults chosen by measurement on the named workloads
 #ifndef TATTN_KS_128B
 #define TATTN_KS_128B 2
@@ -188,6 +190,9 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// exp2_poly on a pair, with packed f32x2 arithmetic (10 issue slots per pair instead of 16).
+__device__ __forceinline__ float2 exp2_poly2(float2 x);
+
 __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool fp16) {
   if (fp16) {
     __half2 h = __floats2half2_rn(lo, hi);
@@ -226,6 +231,20 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 //   operand); l accumulates the unrounded p; O is rescaled in TMEM when the max moved.
 // MASKED: keys at tile columns >= lim are invisible (causal diagonal or past N): their x is
 // -inf, so p = 2^-inf = 0 exactly (these tiles use MUFU ex2 for every column).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 n = fadd2(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);  // x - n, exact
+  float2 p = ffma2(make_float2(5.517166853e-02f, 5.517166853e-02f), f,
+                   make_float2(2.426111251e-01f, 2.426111251e-01f));
+  p = ffma2(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
+  p = ffma2(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 template <int D, bool INT8, bool FP16, bool MASKED>
 __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc, int lim, int j, float& m_run,
                                              float& l_run, uint64_t* o_done_t, volatile int* abort_flag) {
@@ -281,8 +300,9 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
       const float2 a = ffma2(xv, sc2, cst2);
       float p0, p1;
       if (!MASKED && (col & 15) >= 16 - C::POLY_PER_16) {
-        p0 = exp2_poly(a.x);
-        p1 = exp2_poly(a.y);
+        const float2 pp = exp2_poly2(a);
+        p0 = pp.x;
+        p1 = pp.y;
       } else {
         p0 = ex2_approx(a.x);
         p1 = ex2_approx(a.y);
