@@ -38,7 +38,7 @@ from attn_workloads import WORKLOADS, make_inputs  # noqa: E402
 
 
 KERNEL_SOURCES = ("tiled_attention_22_b200/csrc/attn_fwd_kernels.cuh", "tiled_attention_22_b200/csrc/ptx.cuh",
-                  "tiled_attention_22_b200/csrc/api.cu")
+                  "tiled_attention_22_b200/csrc/attn_fwd_launch.cuh", "tiled_attention_22_b200/csrc/tma_host.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_kernel_traffic_mha_causal_b4_h32_n4096_d128.txt")
 
 

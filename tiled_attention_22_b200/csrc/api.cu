@@ -48,121 +48,8 @@ int check_shape(int B, int Hq, int Hkv, int N, int d) {
   return ATTN_OK;
 }
 
-// ----------------------------------------- TMA descriptors ----------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-// [BH, N, d] view of a [B, H, N, d] tensor; box = box_x elements x 128 rows x 1 head.
-int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
-             int box_x, CUtensorMapSwizzle swz) {
-  auto fn = encode_fn();
-  if (!fn) {
-    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
-    return ATTN_ERR_LAUNCH;
-  }
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)d * elem_bytes, (cuuint64_t)N * d * elem_bytes};
-  cuuint32_t box[3] = {(cuuint32_t)box_x, 128u, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
-    return ATTN_ERR_LAUNCH;
-  }
-  return ATTN_OK;
-}
-
-CUtensorMapSwizzle swizzle_for(int row_bytes) {
-  return row_bytes >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-}
-
-// ----------------------------------------- fused kernel launch ------------------------------------
-#ifndef TATTN_SPLIT
-#define TATTN_SPLIT 0
-#endif
-
-template <int D, bool INT8, bool FP16>
-int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p, cudaStream_t stream) {
-  using C = FwdCfg<D, INT8>;
-  constexpr bool SPLIT = TATTN_SPLIT != 0;
-  using R = FwdRoles<SPLIT>;
-  CUtensorMap tq, tk, tv;
-  const CUtensorMapDataType qk_dt =
-      INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : (FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
-  const CUtensorMapDataType v_dt = FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  int rc;
-  if ((rc = make_map(&tq, q, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hq, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
-  if ((rc = make_map(&tk, k, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hkv, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
-  if ((rc = make_map(&tv, v, v_dt, 2, D, p.N, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-  auto kern = attn_fwd_kernel<D, INT8, FP16, SPLIT>;
-  // Once per device: allow the dynamic shared memory, and check the register split.  The kernel
-  // moves registers between warpgroups with setmaxnreg; the increase only completes if the
-  // registers the CTA is launched with cover the split, so refuse to launch otherwise.
-  static std::atomic<int> checked[kMaxDevices];
-  int dev = 0;
-  TATTN_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_LAUNCH;
-  if (checked[dev].load(std::memory_order_acquire) != 1) {
-    TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-    cudaFuncAttributes attr;
-    TATTN_CUDA(cudaFuncGetAttributes(&attr, kern));
-    if ((long long)attr.numRegs * R::kThreads <
-            128LL * (R::kSoftmaxWarps / 4 * R::kRegsSoftmax + R::kRegsProducer) ||
-        attr.maxThreadsPerBlock < R::kThreads) {
-      std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
-                    "fused kernel built with %d registers/thread: too few for its register split", attr.numRegs);
-      return ATTN_ERR_LAUNCH;
-    }
-    checked[dev].store(1, std::memory_order_release);
-  }
-  const long long grid = (long long)p.n_mblocks * p.B * p.Hq;
-  kern<<<(unsigned)grid, R::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-  TATTN_CUDA(cudaGetLastError());
-  return ATTN_OK;
-}
-
-template <bool INT8>
-int launch_fwd(const void* q, const void* k, const void* v, int d, int dtype, const FwdParams& p,
-               cudaStream_t stream) {
-  const bool fp16 = dtype == ATTN_FP16;
-  if (d == 128) return fp16 ? launch_fwd_t<128, INT8, true>(q, k, v, p, stream) : launch_fwd_t<128, INT8, false>(q, k, v, p, stream);
-  return fp16 ? launch_fwd_t<64, INT8, true>(q, k, v, p, stream) : launch_fwd_t<64, INT8, false>(q, k, v, p, stream);
-}
-
-FwdParams make_params(int B, int Hq, int Hkv, int N, int causal, float scale, void* o, float* lse) {
-  FwdParams p{};
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.N = N;
-  p.causal = causal;
-  p.n_mblocks = (N + 255) / 256;
-  // Scheduling sections: kv heads whose K and V (16-bit, d=128, the larger case) take at most
-  // TATTN_L2_SECTION_MB (a quarter of the 126 MB L2 by default).
-#ifndef TATTN_L2_SECTION_MB
-#define TATTN_L2_SECTION_MB 32
-#endif
-  const long long kv_bytes = 2LL * N * 128 * 2;
-  long long sec = ((long long)TATTN_L2_SECTION_MB << 20) / (kv_bytes > 0 ? kv_bytes : 1);
-  if (sec < 1) sec = 1;
-  if (sec > (long long)B * Hkv) sec = (long long)B * Hkv;
-  p.sec_kv = (int)sec;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.o = o;
-  p.lse = lse;
-  return p;
-}
+#include "tma_host.cuh"
+#include "attn_fwd_launch.cuh"
 
 int check_common(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int Hq,
                  int Hkv, int N, int d, int causal, float scale, int dtype) {
