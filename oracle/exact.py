@@ -7,6 +7,9 @@ Follows:
   * same page, section 3.2 (heads are independent) and section 5.1 (a group
     of query heads shares one K/V head).  The grouping is read as contiguous:
     query head h uses kv head h // (Hq / Hkv).
+  * same page, section 3.4 (KV cache: the keys and values of earlier tokens are kept and each
+    new token's query attends to all of them), which fixes the causal alignment of Nq < Nk
+    query rows: they are the last Nq positions;
   * "FlashAttention" glossary page (aiunderstanding.org), FAQ: FlashAttention
     computes exactly the values of standard attention, only reordered, so the
     plain definition is the reference for the tiled kernel.
@@ -38,11 +41,17 @@ def _kv_head(h: int, Hq: int, Hkv: int) -> int:
 
 
 def _scores(qh, kh, scale, causal, rows):
-    """Scaled scores of the selected query rows against all keys, masked."""
+    """Scaled scores of the selected query rows against all keys, masked.
+
+    With Nq query rows and Nk keys, query row i sits at position Nk - Nq + i (the queries are
+    the last Nq tokens, as when a KV cache holds the earlier ones); under the causal mask it
+    sees keys j <= Nk - Nq + i.  With Nq = Nk this is the usual j <= i.
+    """
     S = scale * (qh[rows] @ kh.T)
     if causal:
+        offset = kh.shape[0] - qh.shape[0]
         j = np.arange(kh.shape[0])[None, :]
-        S = np.where(j > np.asarray(rows)[:, None], -np.inf, S)
+        S = np.where(j > np.asarray(rows)[:, None] + offset, -np.inf, S)
     return S
 
 
@@ -65,7 +74,8 @@ def logsumexp_rows(S):
 def attention(q, k, v, scale, causal, rows=None):
     """O = softmax(scale*Q K^T [+causal mask]) V and lse, in float64.
 
-    q: [B, Hq, N, d]; k, v: [B, Hkv, N, d].  ``rows`` optionally restricts the
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] (Nq = Nk for self-attention; Nq < Nk for
+    queries that follow Nk - Nq cached tokens, see _scores).  ``rows`` optionally restricts the
     query rows (each row is independent, so a subset is exact for those rows).
     Returns (O [B, Hq, R, d], lse [B, Hq, R]).
     """

@@ -51,16 +51,17 @@ def test_hand_cases_n4(golden_dir):
 
 
 def _brute(q, k, v, scale, causal):
-    """Pure-Python loops with math.exp: no numpy, no matmul."""
+    """Pure-Python loops with math.exp: no numpy, no matmul.  Query i of Nq is token
+    Nk - Nq + i (the last Nq tokens), so causally it sees keys 0 .. Nk - Nq + i."""
     B, Hq, N, d = q.shape
-    Hkv = k.shape[1]
+    Hkv, Nk = k.shape[1], k.shape[2]
     O = np.zeros((B, Hq, N, v.shape[3]))
     L = np.zeros((B, Hq, N))
     for b in range(B):
         for h in range(Hq):
             g = h // (Hq // Hkv)
             for i in range(N):
-                js = range(i + 1) if causal else range(N)
+                js = range(Nk - N + i + 1) if causal else range(Nk)
                 s = [scale * sum(float(q[b, h, i, c]) * float(k[b, g, j, c]) for c in range(d)) for j in js]
                 m = max(s)
                 w = [math.exp(x - m) for x in s]
@@ -201,3 +202,46 @@ def test_byte_and_flop_figures_from_the_pages():
     B, H, N, d = 1, 2, 128, 64
     assert attention_flops(B, H, N, d, False) == 2 * (2 * B * H * N * N * d)
     assert attention_flops(B, H, N, d, True) == attention_flops(B, H, N, d, False) / 2
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nk", [(1, 9), (3, 11), (5, 5)])
+def test_brute_force_short_queries(causal, Nq, Nk):
+    """Queries that follow a KV cache: Nq < Nk, bottom-right causal alignment."""
+    q = RNG.standard_normal((1, 4, Nq, 6))
+    k = RNG.standard_normal((1, 2, Nk, 6))
+    v = RNG.standard_normal((1, 2, Nk, 3))
+    O, L = oracle.attention(q, k, v, 0.5, causal)
+    Ob, Lb = _brute(q, k, v, 0.5, causal)
+    np.testing.assert_allclose(O, Ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L, Lb, rtol=0, atol=1e-12)
+
+
+def test_short_queries_match_torch_sdpa_with_explicit_mask():
+    """Library cross-check for Nq < Nk: torch's SDPA with an explicit bottom-right causal mask
+    (its own is_causal aligns top-left, so the mask is passed)."""
+    g = torch.Generator().manual_seed(11)
+    Nq, Nk = 7, 300
+    q = torch.randn(2, 8, Nq, 64, generator=g, dtype=torch.float64)
+    k = torch.randn(2, 2, Nk, 64, generator=g, dtype=torch.float64)
+    v = torch.randn(2, 2, Nk, 64, generator=g, dtype=torch.float64)
+    mask = torch.arange(Nk)[None, :] <= (torch.arange(Nq)[:, None] + Nk - Nq)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q, k.repeat_interleave(4, dim=1), v.repeat_interleave(4, dim=1), attn_mask=mask, scale=0.125)
+    O, _ = oracle.attention(q, k, v, 0.125, True)
+    np.testing.assert_allclose(O, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_short_queries_equal_the_last_rows_of_full_self_attention():
+    """The last Nq rows of Nk x Nk causal self-attention are the Nq-query problem over the same
+    keys; a single query (Nq = 1) sees every key, with or without the mask."""
+    q = RNG.standard_normal((1, 2, 40, 8))
+    k = RNG.standard_normal((1, 2, 40, 8))
+    v = RNG.standard_normal((1, 2, 40, 8))
+    O, L = oracle.attention(q, k, v, 0.3, True)
+    Os, Ls = oracle.attention(q[:, :, -6:], k, v, 0.3, True)
+    np.testing.assert_array_equal(Os, O[:, :, -6:])
+    np.testing.assert_array_equal(Ls, L[:, :, -6:])
+    O1c, _ = oracle.attention(q[:, :, -1:], k, v, 0.3, True)
+    O1n, _ = oracle.attention(q[:, :, -1:], k, v, 0.3, False)
+    np.testing.assert_array_equal(O1c, O1n)
