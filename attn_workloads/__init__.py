@@ -26,7 +26,8 @@ import math
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "attention_flops", "workload"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "attention_flops", "workload", "DecodeWorkload",
+           "DECODE_WORKLOADS", "make_decode_inputs", "decode_bytes"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -110,3 +111,80 @@ def make_inputs(w: Workload):
         raise ValueError(f"unknown input kind {w.kind!r}")
     dt = w.torch_dtype
     return q.to(dt), k.to(dt), v.to(dt)
+
+
+# ------------------------------------------------------------------------------------------------
+# KV-cache decoding: Nq new tokens per sequence against a cache of capacity Nk.
+#
+# Recipe: as above (q, k, v i.i.d. N(0, 1) drawn in float32 with seeds seed_base + {0, 1, 2},
+# "k_offset" adds the per-channel N(0, 3^2) offset with seed seed_base + 3, then cast), with the
+# cache drawn at full capacity Nk.  Lengths: "full" gives every sequence Nk cached keys; "ragged"
+# draws kv_lens[b] uniformly from [Nk/2, Nk] with seed seed_base + 4.
+# ------------------------------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    dtype: str
+    kind: str
+    lens: str           # "full" | "ragged"
+    seed_base: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def torch_dtype(self):
+        return {"bf16": torch.bfloat16, "fp16": torch.float16}[self.dtype]
+
+    def replace(self, **kw) -> "DecodeWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+# 101: one decoding step of a LLaMA-3-8B-shaped GQA layer (32 query heads, 8 kv heads, d = 128)
+#      for 8 sequences at 32K context: 1 GiB of cache.
+# 102: the same for an MHA layer of the LLaMA-7B shape (32 heads x 128: 16 KB of K and V per token
+#      and layer in 16-bit) for 16 sequences at 8K context: 2 GiB of cache.
+# 103: verifying 4 drafted tokens (causal among themselves) over ragged lengths up to 16K.
+DECODE_WORKLOADS = {
+    101: DecodeWorkload("gqa_decode_b8_hq32_hkv8_nq1_nk32768_d128", 8, 32, 8, 1, 32768, 128, False, "bf16",
+                        "normal", "full", 101000),
+    102: DecodeWorkload("mha_decode_b16_h32_nq1_nk8192_d128", 16, 32, 32, 1, 8192, 128, False, "bf16",
+                        "normal", "full", 102000),
+    103: DecodeWorkload("gqa_verify_b4_hq32_hkv8_nq4_nk16384_ragged_causal", 4, 32, 8, 4, 16384, 128, True,
+                        "bf16", "k_offset", "ragged", 103000),
+}
+
+
+def make_decode_inputs(w: DecodeWorkload):
+    """Return (q, k_cache, v_cache, kv_lens) as CPU tensors; kv_lens is int32 [B]."""
+    f32 = torch.float32
+    q = torch.randn((w.B, w.Hq, w.Nq, w.d), generator=_gen(w.seed_base + 0), dtype=f32)
+    k = torch.randn((w.B, w.Hkv, w.Nk, w.d), generator=_gen(w.seed_base + 1), dtype=f32)
+    v = torch.randn((w.B, w.Hkv, w.Nk, w.d), generator=_gen(w.seed_base + 2), dtype=f32)
+    if w.kind == "k_offset":
+        k.add_(torch.randn((w.B, w.Hkv, 1, w.d), generator=_gen(w.seed_base + 3), dtype=f32) * 3.0)
+    elif w.kind != "normal":
+        raise ValueError(f"unknown input kind {w.kind!r}")
+    if w.lens == "full":
+        lens = torch.full((w.B,), w.Nk, dtype=torch.int32)
+    elif w.lens == "ragged":
+        lens = torch.randint(w.Nk // 2, w.Nk + 1, (w.B,), generator=_gen(w.seed_base + 4), dtype=torch.int32)
+    else:
+        raise ValueError(f"unknown length rule {w.lens!r}")
+    dt = w.torch_dtype
+    return q.to(dt), k.to(dt), v.to(dt), lens
+
+
+def decode_bytes(B: int, Hq: int, Hkv: int, Nq: int, d: int, lens) -> float:
+    """Algorithmic HBM bytes of one decoding call in 16-bit: the used cache (K and V, sum of the
+    lengths x Hkv x d each), the queries and the outputs; every byte once."""
+    total_len = float(sum(int(x) for x in lens))
+    return 2.0 * 2.0 * total_len * Hkv * d + 2.0 * 2.0 * B * Hq * Nq * d

@@ -179,6 +179,37 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
                   int dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * attn_decode - attention of Nq new query tokens per sequence against a KV cache (decoding, or
+ * verifying a few drafted tokens).  "注意力即一切：从 MHA 到 GQA", section 3.4: with a KV cache the
+ * keys and values of earlier tokens are stored, and each new token's query attends to all of
+ * them; sections 2.2, 2.3 and 5.1 as above for the softmax, the mask and the head grouping.
+ *
+ *   q       [B, Hq, Nq, d]       the new tokens' queries (16-bit, dtype)
+ *   k_cache [B, Hkv, Nk, d]      cached keys; sequence b uses its first kv_lens[b] positions
+ *   v_cache [B, Hkv, Nk, d]      cached values, same layout
+ *   kv_lens device int32 [B], or NULL (every sequence holds Nk keys).  Values are clamped to
+ *           [0, Nk].  Cache entries at or past kv_lens[b] are never used, whatever they hold.
+ *   o       [B, Hq, Nq, d]       output (dtype);  lse  [B, Hq, Nq] float (natural log) or NULL.
+ *   causal  0: every new token sees all kv_lens[b] keys.  1: the new tokens are the LAST Nq of
+ *           the kv_lens[b] positions, so token i sees keys 0 .. kv_lens[b] - Nq + i.  A row that
+ *           sees no key (kv_lens[b] = 0, or kv_lens[b] < Nq under the mask) gets O = 0 and
+ *           lse = -inf.
+ *   d must be 128 and (Hq / Hkv) * Nq <= 64 (ATTN_ERR_UNSUPPORTED otherwise); 1 <= Nq <= Nk.
+ *   num_splits: CTAs per (batch, kv head) along the key range (split-KV).  0 picks a count from
+ *           the shape and the current device's SM count; a positive count is capped at the
+ *           number of 128-key tiles.  More than one split needs `workspace` of at least
+ *           attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits) bytes (16-byte
+ *           aligned; its contents need no initialisation) and launches a second, small kernel
+ *           that merges the splits by their log-sum-exp.
+ *   kv_lens must be 4-byte aligned; every other pointer 16-byte aligned.
+ */
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits);
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens,
+                void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                float scale, int dtype, int num_splits, void* workspace, size_t ws_bytes,
+                void* stream);
+
+/*
  * attn_check_status - synchronises the current device, returns ATTN_OK or
  * ATTN_ERR_TIMEOUT if a device-side wait ran out since the last call, and
  * clears the status word.

@@ -14,6 +14,8 @@ from .binding import (  # noqa: F401
     AttnError,
     LIB_PATH,
     attn_check_status,
+    attn_decode,
+    attn_decode_workspace_bytes,
     attn_error_string,
     attn_fwd,
     attn_fwd_host,

@@ -39,6 +39,8 @@ _SIGNATURES = {
     "attn_probe_qk_int32": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp]),
     "attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i,
                            _vp, _sz, _vp]),
+    "attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _sz, _vp]),
+    "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "attn_check_status": (_i, []),
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_last_cuda_error": (ctypes.c_char_p, []),
@@ -138,6 +140,43 @@ def attn_fwd(q, k, v, causal=False, scale=None, mode="bf16_exact", out=None, lse
                       MODES[mode], DTYPES[q.dtype], _ptr(workspace),
                       0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "attn_fwd")
+    return o, l
+
+
+def attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits=0) -> int:
+    return int(load_library().attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits))
+
+
+def attn_decode(q, k_cache, v_cache, kv_lens=None, causal=False, scale=None, num_splits=0, out=None, lse=True,
+                workspace=None, stream=None):
+    """Attention of q [B, Hq, Nq, d] against the first kv_lens[b] keys of k_cache / v_cache
+    [B, Hkv, Nk, d] (kv_lens: int32 CUDA tensor [B] or None for all Nk).  Returns (o, lse or None)."""
+    lib = load_library()
+    if q.dim() != 4 or k_cache.dim() != 4 or v_cache.dim() != 4:
+        raise ValueError("q, k_cache, v_cache must be [B, H, N, d]")
+    B, Hq, Nq, d = q.shape
+    if k_cache.shape != v_cache.shape or k_cache.shape[0] != B or k_cache.shape[3] != d:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k_cache.shape)} v {tuple(v_cache.shape)}")
+    Hkv, Nk = k_cache.shape[1], k_cache.shape[2]
+    for t in (q, k_cache, v_cache):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k_cache, v_cache must be contiguous CUDA tensors")
+    if q.dtype not in DTYPES or k_cache.dtype != q.dtype or v_cache.dtype != q.dtype:
+        raise ValueError("q, k_cache, v_cache must share one dtype: bfloat16 or float16")
+    if kv_lens is not None and (kv_lens.dtype != torch.int32 or not kv_lens.is_cuda or kv_lens.numel() != B
+                                or not kv_lens.is_contiguous()):
+        raise ValueError("kv_lens must be a contiguous int32 CUDA tensor of B entries")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    l = _lse_arg(lse, (B, Hq, Nq), q.device)
+    ws_bytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    rc = lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kv_lens), _ptr(o), _ptr(l), B, Hq, Hkv, Nq,
+                         Nk, d, int(bool(causal)), scale, DTYPES[q.dtype], int(num_splits), _ptr(workspace),
+                         0 if workspace is None else workspace.numel() * workspace.element_size(),
+                         _stream(stream))
+    _check(rc, "attn_decode")
     return o, l
 
 

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -15,6 +16,7 @@
 #include "tiled_attention.h"
 
 #include "attn_fwd_kernels.cuh"
+#include "decode_kernels.cuh"
 #include "prepass_kernels.cuh"
 
 namespace {
@@ -50,6 +52,7 @@ int check_shape(int B, int Hq, int Hkv, int N, int d) {
 
 #include "tma_host.cuh"
 #include "attn_fwd_launch.cuh"
+#include "decode_launch.cuh"
 
 int check_common(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int Hq,
                  int Hkv, int N, int d, int causal, float scale, int dtype) {
@@ -408,6 +411,51 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   return ATTN_OK;
 }
 
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {
+  if (check_decode_shape(B, Hq, Hkv, Nq, Nk, d, num_splits)) return 0;
+  return decode_ws(B, Hq, Nq, decode_splits(B, Hkv, Nk, num_splits)).total;
+}
+
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens, void* o, float* lse,
+                int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale, int dtype, int num_splits,
+                void* workspace, size_t ws_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !o) return ATTN_ERR_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_ARG;
+  int rc = check_decode_shape(B, Hq, Hkv, Nq, Nk, d, num_splits);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || (lse && !aligned16(lse)) ||
+      (reinterpret_cast<uintptr_t>(kv_lens) & 3u))
+    return ATTN_ERR_ALIGN;
+  const int nsplit = decode_splits(B, Hkv, Nk, num_splits);
+  if ((long long)B * Hkv * nsplit > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;  // grid x extent
+  const DecWs w = decode_ws(B, Hq, Nq, nsplit);
+  if (w.total > 0) {
+    if (!workspace || ws_bytes < w.total) return ATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
+  }
+  DecParams p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.R = (Hq / Hkv) * Nq;
+  p.causal = causal;
+  p.nsplit = nsplit;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.kv_lens = kv_lens;
+  p.o = o;
+  p.lse = lse;
+  if (w.total > 0) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.part_o = reinterpret_cast<float*>(ws + w.part_o);
+    p.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
+  }
+  return launch_decode(q, k_cache, v_cache, dtype, p, static_cast<cudaStream_t>(stream));
+}
+
 int attn_check_status(void) {
   TATTN_CUDA(cudaDeviceSynchronize());
   int st = 0, zero = 0;
@@ -438,7 +486,7 @@ const char* attn_error_string(int code) {
   switch (code) {
     case ATTN_OK: return "ok";
     case ATTN_ERR_ARG: return "invalid argument";
-    case ATTN_ERR_UNSUPPORTED: return "unsupported size (d must be 64 or 128)";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported size (d must be 64 or 128; decode: d = 128, (Hq/Hkv)*Nq <= 64)";
     case ATTN_ERR_ALIGN: return "device pointer not 16-byte aligned";
     case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
     case ATTN_ERR_LAUNCH: return "CUDA launch or call failed";

@@ -1,0 +1,470 @@
+// decode_kernels.cuh - attention of a few new query tokens against a KV cache (decode / short-query
+// forward), for sm_100a.
+//
+// What it computes: for every (batch b, query head h) and each of the Nq new tokens i,
+// O = softmax(scale * q K^T [+ causal mask]) V over the first len_b cached keys of kv head
+// h / (Hq/Hkv) ("注意力即一切：从 MHA 到 GQA", section 3.4: with a KV cache each new token's query
+// attends to the stored keys and values of all earlier tokens; sections 2.2, 2.3 and 5.1 for the
+// softmax, the mask and the head grouping).  The new tokens are the last Nq of the len_b, so under
+// the causal mask token i sees keys 0 .. len_b - Nq + i.
+//
+// Why a second kernel: decoding reads the whole cache for a handful of query rows, so it is bound
+// by HBM bandwidth, not by the tensor core.  The prefill kernel's 128-row query tiles would be
+// almost empty, and it would read each kv head's cache once per query head.
+//
+// B200 design:
+//   * One CTA per (batch, kv head, split of the key range): all G = Hq/Hkv query heads x Nq tokens
+//     of that kv head (R = G * Nq rows, padded to RP = 16, 32 or 64) are served by one pass over
+//     the cache, so every cached byte is read once (GQA-aware).  The key range of a sequence is
+//     split across CTAs (split-KV) so that small batches still put enough SMs on the cache; the
+//     splits are merged by their log-sum-exp in a second small kernel.
+//   * The score tile is computed transposed, S^T = K Q^T (tcgen05.mma, M = 128 keys, N = RP query
+//     rows): TMEM lane = key.  Each softmax thread owns one key and RP/NWG query columns; the
+//     column maxima over the 128 keys take one redux.sync per column and warp plus a 4-warp
+//     exchange in shared memory.  P^T is written to shared memory (16-bit, 128-byte swizzle) and
+//     O^T += V^T P^T is a second MMA whose A operand is the V tile read MN-major, so TMEM lane =
+//     output channel.  The row sums l stay per thread (per key lane) and are reduced once at the
+//     end.
+//   * K and V tiles (128 keys x 128 channels) stream through TMA rings with evict-first hints; the
+//     next tile's S^T is computed while the softmax works on the current one (two S^T buffers).
+//   * Cache entries past len_b are never used: their scores are masked and, in the last tile of a
+//     sequence, their V rows are zeroed in shared memory before the P V product, so whatever the
+//     cache holds there (NaN included) cannot reach the output.
+//   * Lazy rescaling as in the prefill kernel (the running max moves only when a column's max
+//     grows by more than 2^8), bounded waits everywhere, and a group-wide AND at every named
+//     barrier so that a timeout makes all threads of a warpgroup leave together.
+#pragma once
+#include <climits>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace tattn {
+
+struct DecParams {
+  int B, Hq, Hkv, Nq, Nk;
+  int R;                 // (Hq / Hkv) * Nq query rows per kv head
+  int causal;
+  int nsplit;            // CTAs per (batch, kv head)
+  float scale_log2;      // scale * log2(e)
+  const int* kv_lens;    // [B] cached keys per sequence (clamped to [0, Nk]); null: all Nk
+  void* o;               // nsplit == 1: [B, Hq, Nq, 128] 16-bit
+  float* lse;            // nsplit == 1: [B, Hq, Nq] or null
+  float* part_o;         // nsplit > 1: [nsplit, B*Hq*Nq, 128] fp32, normalised per split
+  float* part_lse;       // nsplit > 1: [nsplit, B*Hq*Nq]
+};
+
+template <int RP>
+struct DecCfg {
+  static constexpr int D = 128;
+  static constexpr int CW = RP < 32 ? RP : 32;   // query columns per softmax thread
+  static constexpr int NWG = RP / CW;            // softmax warpgroups
+  static constexpr int kSoftmaxWarps = 4 * NWG;
+  static constexpr int kTmaWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+  static constexpr int PANEL = 128 * 128;        // 128 keys x 64 channels x 2 B (one TMA box)
+  static constexpr int KV_TILE = 2 * PANEL;
+  static constexpr int Q_PANEL = RP * 128, Q_TILE = 2 * Q_PANEL;
+  static constexpr int P_PANEL = RP * 128, P_TILE = 2 * P_PANEL;  // RP rows x 64 keys x 2 B per panel
+  static constexpr int KS = 3;
+  static constexpr int VS = RP <= 32 ? 3 : 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_P = OFF_Q + Q_TILE;
+  static constexpr int OFF_K = OFF_P + 2 * P_TILE;
+  static constexpr int OFF_V = OFF_K + KS * KV_TILE;
+  static constexpr int OFF_RED = OFF_V + VS * KV_TILE;    // float [2][RP][4]: per-warp column maxima
+  static constexpr int OFF_LRED = OFF_RED + 2 * RP * 16;  // float [RP][4]: per-warp row sums
+  static constexpr int OFF_M = OFF_LRED + RP * 16;        // float [2][RP]: running column maxima
+  static constexpr int OFF_BAR = OFF_M + 2 * RP * 4;
+  // q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2], o_done,
+  // o_final, drain
+  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 4 + 3;
+  static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
+  static constexpr int SMEM_BYTES = SMEM_USED + 1024;
+  static constexpr uint32_t TMEM_COLS = 3 * RP <= 64 ? 64u : (3 * RP <= 128 ? 128u : 256u);
+  __host__ __device__ static constexpr uint32_t tm_s(int buf) { return (uint32_t)(buf * RP); }
+  static constexpr uint32_t TM_O = 2 * RP;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(RP % 16 == 0 && RP <= 64, "N of the M = 128 MMAs");
+};
+
+enum : int { WD_LOAD = 0x60, WD_MMA = 0x70, WD_SOFTMAX = 0x80, WD_DRAIN = 0x90 };
+
+// S^T(tmem, 128 keys x RP) = K_tile (128 x 128, K-major) * Q^T (Q: RP x 128, K-major); both staged
+// by TMA with the 128-byte swizzle in two 64-channel panels.
+template <int RP, bool FP16>
+__device__ __forceinline__ void issue_kq(uint32_t s_tmem, uint32_t k_smem, uint32_t q_smem) {
+  constexpr uint32_t idesc = instr_desc(1, FP16 ? 0 : 1, 0, 0, 128, RP);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {  // 16 channels (32 bytes) per MMA
+    const uint32_t col = (uint32_t)(kk & 3) * 32;
+    const uint64_t ad = smem_desc(k_smem + (kk >> 2) * DecCfg<RP>::PANEL + col, 16, 1024, kSwizzle128B);
+    const uint64_t bd = smem_desc(q_smem + (kk >> 2) * DecCfg<RP>::Q_PANEL + col, 16, 1024, kSwizzle128B);
+    mma_f16_ss(s_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O^T(tmem, 128 channels x RP) (+)= V^T (V_tile read MN-major: 64-channel panels 16 KB apart,
+// 8-key groups 1024 B apart) * P^T (P: RP x 128 keys, K-major, two 64-key panels).
+template <int RP, bool FP16>
+__device__ __forceinline__ void issue_vp(uint32_t o_tmem, uint32_t v_smem, uint32_t p_smem, bool accumulate) {
+  constexpr uint32_t idesc = instr_desc(1, FP16 ? 0 : 1, 1, 0, 128, RP);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {  // 16 keys per MMA
+    const uint64_t ad = smem_desc(v_smem + kk * 16 * 128, DecCfg<RP>::PANEL, 1024, kSwizzle128B);
+    const uint64_t bd =
+        smem_desc(p_smem + (kk >> 2) * DecCfg<RP>::P_PANEL + (uint32_t)(kk & 3) * 32, 16, 1024, kSwizzle128B);
+    mma_f16_ss(o_tmem, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <bool FP16>
+__device__ __forceinline__ uint16_t to16(float x) {
+  if constexpr (FP16) return __half_as_ushort(__float2half_rn(x));
+  else return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+template <int CW>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CW]) {
+  if constexpr (CW == 16) {
+    tmem_ld16(taddr, r);
+    tmem_ld_wait16(r);
+  } else {
+    tmem_ld32(taddr, r);
+    tmem_ld_wait(r);
+  }
+}
+template <int CW>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[CW]) {
+  if constexpr (CW == 16) tmem_st16(taddr, r);
+  else tmem_st32(taddr, r);
+}
+
+template <int RP, bool FP16>
+__global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
+    attn_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const DecParams p) {
+  using C = DecCfg<RP>;
+  constexpr int CW = C::CW;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = q_full + 1;
+  uint64_t* k_empty = k_full + C::KS;
+  uint64_t* v_full = k_empty + C::KS;
+  uint64_t* v_empty = v_full + C::VS;
+  uint64_t* s_full = v_empty + C::VS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* o_final = o_done + 1;
+  uint64_t* drain = o_final + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sP = smem + C::OFF_P;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  float* lred = reinterpret_cast<float*>(smem + C::OFF_LRED);
+  float* m_sh = reinterpret_cast<float*>(smem + C::OFF_M);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < C::KS; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+    for (int i = 0; i < C::VS; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], C::kSoftmaxWarps); }
+    mbar_init(o_done, 1);
+    mbar_init(o_final, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::kMmaWarp) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == C::kTmaWarp && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // ---- work item: (batch, kv head) x split of that sequence's key tiles ----
+  const int bkv = (int)(blockIdx.x / (unsigned)p.nsplit);
+  const int split = (int)blockIdx.x - bkv * p.nsplit;
+  const int b = bkv / p.Hkv;
+  int len = p.kv_lens ? __ldg(&p.kv_lens[b]) : p.Nk;
+  len = min(max(len, 0), p.Nk);
+  const int ntiles = (len + 127) / 128;
+  const int chunk = (ntiles + p.nsplit - 1) / p.nsplit;
+  const int t_lo = min(split * chunk, ntiles);
+  const int nt = min(t_lo + chunk, ntiles) - t_lo;
+
+  if (warp == C::kTmaWarp) {
+    // ================================ TMA producer ================================
+    if (lane == 0 && nt > 0) {
+      const uint64_t pol = policy_evict_first();  // every cached byte is read once
+      int k_issued = 0, v_issued = 0;
+      bool ok = true;
+      mbar_arrive_expect_tx(q_full, C::Q_TILE);
+      for (int pn = 0; pn < 2; ++pn) tma_load_3d(sQ + pn * C::Q_PANEL, &tmQ, pn * 64, 0, bkv, q_full, pol);
+      for (int j = 0; j < nt && ok; ++j) {
+        const int ks = j % C::KS, vs = j % C::VS;
+        const int key0 = (t_lo + j) * 128;
+        if (!(ok = mbar_wait(&k_empty[ks], ((j / C::KS) & 1) ^ 1, abort_flag, WD_LOAD + 1))) break;
+        mbar_arrive_expect_tx(&k_full[ks], C::KV_TILE);
+        for (int pn = 0; pn < 2; ++pn)
+          tma_load_3d(sK + ks * C::KV_TILE + pn * C::PANEL, &tmK, pn * 64, key0, bkv, &k_full[ks], pol);
+        k_issued = j + 1;
+        if (!(ok = mbar_wait(&v_empty[vs], ((j / C::VS) & 1) ^ 1, abort_flag, WD_LOAD + 2))) break;
+        mbar_arrive_expect_tx(&v_full[vs], C::KV_TILE);
+        for (int pn = 0; pn < 2; ++pn)
+          tma_load_3d(sV + vs * C::KV_TILE + pn * C::PANEL, &tmV, pn * 64, key0, bkv, &v_full[vs], pol);
+        v_issued = j + 1;
+      }
+      if (!ok) {
+        // every issued copy must land before the CTA's shared memory is released
+        mbar_wait(q_full, 0, nullptr, WD_DRAIN + 1, 200000000ull);
+        for (int j = max(0, k_issued - C::KS); j < k_issued; ++j)
+          mbar_wait(&k_full[j % C::KS], (j / C::KS) & 1, nullptr, WD_DRAIN + 2, 200000000ull);
+        for (int j = max(0, v_issued - C::VS); j < v_issued; ++j)
+          mbar_wait(&v_full[j % C::VS], (j / C::VS) & 1, nullptr, WD_DRAIN + 3, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::kMmaWarp) {
+    // ================================ MMA issuer ================================
+    if (lane == 0 && nt > 0) {
+      const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      bool ok = mbar_wait(q_full, 0, abort_flag, WD_MMA + 1);
+      // S^T of tiles 0 and 1 up front; S^T(j + 2) is issued right after O^T += V^T P^T(j)
+      for (int j = 0; j < 2 && j < nt && ok; ++j) {
+        if (!(ok = mbar_wait(&k_full[j % C::KS], (j / C::KS) & 1, abort_flag, WD_MMA + 2))) break;
+        tc_fence_after();
+        issue_kq<RP, FP16>(tmem + C::tm_s(j), k_addr + (j % C::KS) * C::KV_TILE, q_addr);
+        mma_commit(&s_full[j]);
+        mma_commit(&k_empty[j % C::KS]);
+      }
+      for (int j = 0; j < nt && ok; ++j) {
+        const int vs = j % C::VS;
+        if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, WD_MMA + 3))) break;
+        if (!(ok = mbar_wait(&v_full[vs], (j / C::VS) & 1, abort_flag, WD_MMA + 4))) break;
+        tc_fence_after();
+        issue_vp<RP, FP16>(tmem + C::TM_O, v_addr + vs * C::KV_TILE, p_addr + (j & 1) * C::P_TILE, j > 0);
+        mma_commit(&v_empty[vs]);
+        mma_commit(o_done);  // one phase per tile
+        if (j + 1 == nt) mma_commit(o_final);
+        if (j + 2 < nt) {
+          const int ks = (j + 2) % C::KS;
+          if (!(ok = mbar_wait(&k_full[ks], ((j + 2) / C::KS) & 1, abort_flag, WD_MMA + 5))) break;
+          tc_fence_after();
+          issue_kq<RP, FP16>(tmem + C::tm_s(j & 1), k_addr + ks * C::KV_TILE, q_addr);
+          mma_commit(&s_full[j & 1]);
+          mma_commit(&k_empty[ks]);
+        }
+      }
+      if (!ok) {
+        // every MMA issued so far must complete before TMEM is released
+        mma_commit(drain);
+        mbar_wait(drain, 0, nullptr, WD_DRAIN + 4, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================================ softmax ================================
+    const int wg = warp >> 2, wq = warp & 3;
+    const int t = wq * 32 + lane;    // TMEM lane: key t of the S^T tile, channel t of O^T
+    const int c0 = wg * CW;          // first query column of this warpgroup
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const int bar_id = 1 + wg;
+    const int rows_total = p.B * p.Hkv * p.R;
+    // Keys [0, lim(c)) are visible to query column c: lim = len, or under the causal mask
+    // len - Nq + 1 + (c mod Nq).  Tiles that end at or before `edge` need no mask at all.  Padded
+    // columns (c >= R) are never masked: their Q rows are zeros, they only ever feed their own
+    // columns of O^T and l, and nothing of them is written out.
+    const int causal_base = len - p.Nq + 1;
+    const int edge = p.causal ? min(len, causal_base) : len;
+    // P^T store address of element (row c, key t): two 64-key panels, 128-byte swizzle
+    const uint32_t p_base = smem_u32(sP) + (uint32_t)(t >> 6) * C::P_PANEL + (uint32_t)(t & 7) * 2;
+    const uint32_t p_chunk = (uint32_t)((t & 63) >> 3);
+    float l_run[CW];
+#pragma unroll
+    for (int r = 0; r < CW; ++r) l_run[r] = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int buf = j & 1;
+      bool okw = mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, WD_SOFTMAX + 1);
+      okw = __all_sync(0xffffffffu, okw);
+      float s[CW];
+      const int tile0 = (t_lo + j) * 128;
+      const int key = tile0 + t;
+      if (okw) {
+        tc_fence_after();
+        uint32_t raw[CW];
+        tmem_ld_cols<CW>(tmem + C::tm_s(buf) + (uint32_t)c0 + lane_off, raw);
+#pragma unroll
+        for (int r = 0; r < CW; ++r) s[r] = __uint_as_float(raw[r]);
+        if (tile0 + 128 > edge) {  // (the same for the whole warpgroup)
+#pragma unroll
+          for (int r = 0; r < CW; ++r) {
+            const int c = c0 + r;
+            const int lim = p.causal ? causal_base + c % p.Nq : len;
+            if (c < p.R && key >= lim) s[r] = -INFINITY;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < CW; ++r) s[r] = -INFINITY;
+      }
+#pragma unroll
+      for (int r = 0; r < CW; ++r) {
+        const float wm = warp_max_f32(s[r]);
+        if (lane == 0) red[(buf * RP + c0 + r) * 4 + wq] = wm;
+      }
+      if (!(ok = named_bar_and(bar_id, 128, okw && ok))) break;
+      // Column maxima over the 128 keys and the lazy update of the running max m (kept in shared
+      // memory, double-buffered by tile parity: every thread computes the same m, lane r of the
+      // group's first warp stores column c0 + r).  Then P^T(j) = exp2(s * scale_log2 - m), with
+      // masked keys giving exp2(-inf) = 0, and the per-key partial row sums.
+      float alpha[CW];
+      bool resc = false;
+      const uint32_t pb = p_base + (uint32_t)buf * C::P_TILE;
+#pragma unroll
+      for (int r = 0; r < CW; ++r) {
+        const int c = c0 + r;
+        const float4 w4 = *reinterpret_cast<const float4*>(&red[(buf * RP + c) * 4]);
+        const float mt = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w)) * p.scale_log2;
+        const float m_old = j > 0 ? m_sh[(buf ^ 1) * RP + c] : -INFINITY;
+        const float mn = fmaxf(m_old, mt);
+        float m_use = m_old;
+        alpha[r] = 1.f;
+        if (mn > m_old + 8.f) {
+          alpha[r] = ex2_approx(m_old - mn);
+          m_use = mn;
+          resc = true;
+        }
+        if (wq == 0 && lane == r) m_sh[buf * RP + c] = m_use;
+        const float pv = ex2_approx(fmaf(s[r], p.scale_log2, m_use == -INFINITY ? 0.f : -m_use));
+        l_run[r] = fmaf(l_run[r], alpha[r], pv);
+        st_shared_u16(pb + (uint32_t)c * 128 + ((p_chunk ^ (uint32_t)(c & 7)) << 4), to16<FP16>(pv));
+      }
+      // (resc and j are the same for every thread of the warpgroup)
+      if (resc && j > 0) {
+        // O^T must hold P V of tile j - 1 before it is rescaled.  The waiter is never more than
+        // one phase behind: S^T(j) was issued after P V of tile j - 2, and P V of tile j waits
+        // for this warpgroup's P^T(j).
+        bool oko = mbar_wait(o_done, (j - 1) & 1, abort_flag, WD_SOFTMAX + 2);
+        oko = __all_sync(0xffffffffu, oko);
+        if (oko) {
+          tc_fence_after();
+          uint32_t o[CW];
+          tmem_ld_cols<CW>(tmem + C::TM_O + (uint32_t)c0 + lane_off, o);
+#pragma unroll
+          for (int r = 0; r < CW; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
+          tmem_st_cols<CW>(tmem + C::TM_O + (uint32_t)c0 + lane_off, o);
+          tmem_st_wait();
+        }
+        ok = oko;  // on failure the abort flag is raised: the next wait returns at once
+      }
+      // the sequence's last tile: zero the V rows of keys >= len (never valid cache entries)
+      if (wg == 0 && tile0 + 128 > len) {
+        const int vs = j % C::VS;
+        const bool okv = mbar_wait(&v_full[vs], (j / C::VS) & 1, abort_flag, WD_SOFTMAX + 3);
+        if (okv && key >= len) {
+          const uint32_t vrow = smem_u32(sV) + (uint32_t)vs * C::KV_TILE + (uint32_t)t * 128;
+#pragma unroll
+          for (int pn = 0; pn < 2; ++pn)
+#pragma unroll
+            for (int q16 = 0; q16 < 8; ++q16) st_shared_zero16(vrow + pn * C::PANEL + q16 * 16);
+        }
+        ok = ok && okv;
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[buf]);
+    }
+
+    // ---- epilogue: reduce the row sums over the 128 keys, normalise, write ----
+    bool oke = ok;
+    if (nt > 0 && oke) oke = mbar_wait(o_final, 0, abort_flag, WD_SOFTMAX + 4);
+#pragma unroll
+    for (int r = 0; r < CW; ++r) {
+      float v = l_run[r];
+#pragma unroll
+      for (int sh = 16; sh > 0; sh >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sh);
+      if (lane == 0) lred[(c0 + r) * 4 + wq] = v;
+    }
+    if (named_bar_and(bar_id, 128, oke)) {
+      uint32_t o[CW];
+      if (nt > 0) {
+        tc_fence_after();
+        tmem_ld_cols<CW>(tmem + C::TM_O + (uint32_t)c0 + lane_off, o);
+      } else {
+#pragma unroll
+        for (int r = 0; r < CW; ++r) o[r] = 0u;
+      }
+      const float* m_last = m_sh + ((nt - 1) & 1) * RP;
+#pragma unroll
+      for (int r = 0; r < CW; ++r) {
+        const int c = c0 + r;
+        if (c < p.R) {
+          const float4 l4 = *reinterpret_cast<const float4*>(&lred[c * 4]);
+          const float lsum = (l4.x + l4.y) + (l4.z + l4.w);
+          const float val = lsum > 0.f ? __uint_as_float(o[r]) / lsum : 0.f;
+          const size_t row = (size_t)bkv * p.R + c;
+          float lse = -INFINITY;
+          if (t == r && lsum > 0.f) lse = (m_last[c] + __log2f(lsum)) * 0.69314718055994531f;
+          if (p.nsplit == 1) {
+            reinterpret_cast<uint16_t*>(p.o)[row * 128 + t] = to16<FP16>(val);
+            if (p.lse != nullptr && t == r) p.lse[row] = lse;
+          } else {
+            p.part_o[((size_t)split * rows_total + row) * 128 + t] = val;
+            if (t == r) p.part_lse[(size_t)split * rows_total + row] = lse;
+          }
+        }
+      }
+    }
+    tmem_st_wait();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Merge of the splits of one query row: O = sum_s w_s O_s / sum_s w_s with w_s = exp(lse_s - max),
+// lse = max + log(sum_s w_s).  One CTA of 128 threads (one per channel) per row.
+template <bool FP16>
+__global__ void __launch_bounds__(128) attn_decode_combine_kernel(const float* __restrict__ part_o,
+                                                                  const float* __restrict__ part_lse, int nsplit,
+                                                                  int rows, void* o, float* lse) {
+  const int row = blockIdx.x, c = threadIdx.x;
+  float mx = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, __ldg(&part_lse[(size_t)s * rows + row]));
+  float wsum = 0.f, acc = 0.f;
+  if (mx != -INFINITY) {
+    for (int s = 0; s < nsplit; ++s) {
+      const float ls = __ldg(&part_lse[(size_t)s * rows + row]);
+      const float w = ls == -INFINITY ? 0.f : __expf(ls - mx);
+      wsum += w;
+      acc = fmaf(w, __ldg(&part_o[((size_t)s * rows + row) * 128 + c]), acc);
+    }
+  }
+  const float val = wsum > 0.f ? acc / wsum : 0.f;
+  reinterpret_cast<uint16_t*>(o)[(size_t)row * 128 + c] = to16<FP16>(val);
+  if (lse != nullptr && c == 0) lse[row] = wsum > 0.f ? mx + __logf(wsum) : -INFINITY;
+}
+
+}  // namespace tattn

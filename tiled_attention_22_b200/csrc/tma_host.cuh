@@ -14,9 +14,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [BH, N, d] view of a [B, H, N, d] tensor; box = box_x elements x 128 rows x 1 head.
+// [BH, N, d] view of a [B, H, N, d] tensor; box = box_x elements x box_y rows x 1 head.
 int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int N, int BH,
-             int box_x, CUtensorMapSwizzle swz) {
+             int box_x, CUtensorMapSwizzle swz, int box_y = 128) {
   auto fn = encode_fn();
   if (!fn) {
     std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
@@ -24,7 +24,7 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_
   }
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * elem_bytes, (cuuint64_t)N * d * elem_bytes};
-  cuuint32_t box[3] = {(cuuint32_t)box_x, 128u, 1u};
+  cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
