@@ -74,7 +74,7 @@ struct DecCfg {
   static constexpr int OFF_P = OFF_Q + Q_TILE;
   static constexpr int OFF_K = OFF_P + 2 * P_TILE;
   static constexpr int OFF_V = OFF_K + KS * KV_TILE;
-  static constexpr int OFF_RED = OFF_V + VS * KV_TILE;    // float [2][RP][4]: per-warp column maxima
+  static constexpr int OFF_RED = OFF_V + VS * KV_TILE;    // float [2][4][RP]: per-warp column maxima
   static constexpr int OFF_LRED = OFF_RED + 2 * RP * 16;  // float [RP][4]: per-warp row sums
   static constexpr int OFF_M = OFF_LRED + RP * 16;        // float [2][RP]: running column maxima
   static constexpr int OFF_BAR = OFF_M + 2 * RP * 4;
@@ -324,10 +324,16 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
 #pragma unroll
         for (int r = 0; r < CW; ++r) s[r] = -INFINITY;
       }
+      {
+        float wm[CW];
 #pragma unroll
-      for (int r = 0; r < CW; ++r) {
-        const float wm = warp_max_f32(s[r]);
-        if (lane == 0) red[(buf * RP + c0 + r) * 4 + wq] = wm;
+        for (int r = 0; r < CW; ++r) wm[r] = warp_max_f32(s[r]);
+        if (lane == 0) {
+          float4* dst = reinterpret_cast<float4*>(&red[(buf * 4 + wq) * RP + c0]);
+#pragma unroll
+          for (int q4 = 0; q4 < CW / 4; ++q4)
+            dst[q4] = make_float4(wm[4 * q4], wm[4 * q4 + 1], wm[4 * q4 + 2], wm[4 * q4 + 3]);
+        }
       }
       if (!(ok = named_bar_and(bar_id, 128, okw && ok))) break;
       // Column maxima over the 128 keys and the lazy update of the running max m (kept in shared
@@ -337,24 +343,38 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
       float alpha[CW];
       bool resc = false;
       const uint32_t pb = p_base + (uint32_t)buf * C::P_TILE;
+      const float4* rd = reinterpret_cast<const float4*>(&red[buf * 4 * RP + c0]);
+      const float4* mo = reinterpret_cast<const float4*>(&m_sh[(buf ^ 1) * RP + c0]);
+      float4* mw = reinterpret_cast<float4*>(&m_sh[buf * RP + c0]);
 #pragma unroll
-      for (int r = 0; r < CW; ++r) {
-        const int c = c0 + r;
-        const float4 w4 = *reinterpret_cast<const float4*>(&red[(buf * RP + c) * 4]);
-        const float mt = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w)) * p.scale_log2;
-        const float m_old = j > 0 ? m_sh[(buf ^ 1) * RP + c] : -INFINITY;
-        const float mn = fmaxf(m_old, mt);
-        float m_use = m_old;
-        alpha[r] = 1.f;
-        if (mn > m_old + 8.f) {
-          alpha[r] = ex2_approx(m_old - mn);
-          m_use = mn;
-          resc = true;
+      for (int q4 = 0; q4 < CW / 4; ++q4) {  // four columns at a time: vector loads of the maxima
+        const float4 a = rd[q4], b4 = rd[RP / 4 + q4], c4 = rd[2 * (RP / 4) + q4], d4 = rd[3 * (RP / 4) + q4];
+        const float4 m4 = j > 0 ? mo[q4] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        const float wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b4.x, b4.y, b4.z, b4.w};
+        const float wc[4] = {c4.x, c4.y, c4.z, c4.w}, wd[4] = {d4.x, d4.y, d4.z, d4.w};
+        const float mold[4] = {m4.x, m4.y, m4.z, m4.w};
+        float muse[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 4 * q4 + i;
+          const float mt = fmaxf(fmaxf(wa[i], wb[i]), fmaxf(wc[i], wd[i])) * p.scale_log2;
+          const float mn = fmaxf(mold[i], mt);
+          muse[i] = mold[i];
+          alpha[r] = 1.f;
+          if (mn > mold[i] + 8.f) {
+            alpha[r] = ex2_approx(mold[i] - mn);
+            muse[i] = mn;
+            resc = true;
+          }
         }
-        if (wq == 0 && lane == r) m_sh[buf * RP + c] = m_use;
-        const float pv = ex2_approx(fmaf(s[r], p.scale_log2, m_use == -INFINITY ? 0.f : -m_use));
-        l_run[r] = fmaf(l_run[r], alpha[r], pv);
-        st_shared_u16(pb + (uint32_t)c * 128 + ((p_chunk ^ (uint32_t)(c & 7)) << 4), to16<FP16>(pv));
+        if (wq == 0 && lane == 0) mw[q4] = make_float4(muse[0], muse[1], muse[2], muse[3]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 4 * q4 + i, c = c0 + r;
+          const float pv = ex2_approx(fmaf(s[r], p.scale_log2, muse[i] == -INFINITY ? 0.f : -muse[i]));
+          l_run[r] = fmaf(l_run[r], alpha[r], pv);
+          st_shared_u16(pb + (uint32_t)c * 128 + ((p_chunk ^ (uint32_t)(c & 7)) << 4), to16<FP16>(pv));
+        }
       }
       // (resc and j are the same for every thread of the warpgroup)
       if (resc && j > 0) {

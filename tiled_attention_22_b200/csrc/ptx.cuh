@@ -311,10 +311,11 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
       : "memory");
   return r != 0;
 }
-// Maximum of a float over the 32 lanes of the warp (sm_100a).
+// Maximum of a float over the 32 lanes of the warp (sm_100a).  Not volatile: it has no side
+// effects, so the compiler may overlap several of them.
 __device__ __forceinline__ float warp_max_f32(float x) {
   float r;
-  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  asm("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
   return r;
 }
 // Generic-proxy writes to shared memory (plain stores) made visible to the async proxy
@@ -322,8 +323,11 @@ __device__ __forceinline__ float warp_max_f32(float x) {
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// 16-bit store to a shared-memory operand tile that C++ code never reads: no "memory" clobber,
+// so loads of other shared data can be scheduled across it (volatile asm statements still keep
+// their order, e.g. before a later proxy fence).
 __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v));
 }
 __device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
