@@ -195,18 +195,19 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
  *           sees no key (kv_lens[b] = 0, or kv_lens[b] < Nq under the mask) gets O = 0 and
  *           lse = -inf.
  *   d must be 128 and (Hq / Hkv) * Nq <= 64 (ATTN_ERR_UNSUPPORTED otherwise); 1 <= Nq <= Nk.
- *   num_splits: CTAs per (batch, kv head) along the key range (split-KV).  0 picks a count from
- *           the shape and the current device's SM count; a positive count is capped at the
- *           number of 128-key tiles.  More than one split needs `workspace` of at least
- *           attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits) bytes (16-byte
- *           aligned; its contents need no initialisation) and launches a second, small kernel
- *           that merges the splits by their log-sum-exp.
+ *   num_ctas: persistent CTAs (0: one per SM of the current device).  All key tiles of all
+ *           (batch, kv head) units form one sequence, and CTA i of P takes the contiguous share
+ *           [floor(i T / P), floor((i + 1) T / P)) of its T tiles, so ragged lengths stay
+ *           balanced.  The part of a unit inside one CTA's share is a piece; a second, small
+ *           kernel merges each unit's pieces by their log-sum-exp.
+ *   workspace: at least attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_ctas) bytes,
+ *           16-byte aligned; its contents need no initialisation.
  *   kv_lens must be 4-byte aligned; every other pointer 16-byte aligned.
  */
-size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits);
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas);
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens,
                 void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
-                float scale, int dtype, int num_splits, void* workspace, size_t ws_bytes,
+                float scale, int dtype, int num_ctas, void* workspace, size_t ws_bytes,
                 void* stream);
 
 /*

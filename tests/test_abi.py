@@ -120,30 +120,31 @@ def test_product_package_does_not_import_the_oracle():
 
 
 def _dec(lib, q=FAKE, k=FAKE, v=FAKE, lens=None, o=FAKE, lse=None, B=1, Hq=8, Hkv=2, Nq=1, Nk=1024, d=128,
-         causal=0, scale=0.125, dtype=0, splits=1, ws=None, ws_bytes=0):
-    return lib.attn_decode(q, k, v, lens, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype, splits, ws, ws_bytes,
+         causal=0, scale=0.125, dtype=0, ctas=1, ws=None, ws_bytes=0):
+    return lib.attn_decode(q, k, v, lens, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, dtype, ctas, ws, ws_bytes,
                            None)
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(q=None), -1), (dict(o=None), -1), (dict(Nq=0), -1), (dict(Nq=2000), -1), (dict(Hq=3), -1),
-    (dict(scale=0.0), -1), (dict(causal=-1), -1), (dict(dtype=2), -1), (dict(splits=-1), -1),
+    (dict(scale=0.0), -1), (dict(causal=-1), -1), (dict(dtype=2), -1), (dict(ctas=-1), -1),
     (dict(d=64), -2), (dict(Hq=128, Hkv=1), -2), (dict(Hq=8, Hkv=1, Nq=9), -2),
     (dict(q=FAKE + 2), -3), (dict(lens=FAKE + 2), -3), (dict(lse=FAKE + 8), -3),
-    (dict(splits=4), -4), (dict(splits=4, ws=FAKE, ws_bytes=64), -4),
+    (dict(ctas=4), -4), (dict(ws=FAKE, ws_bytes=64), -4),
 ])
 def test_attn_decode_rejects_bad_arguments(lib, kw, code):
     assert _dec(lib, **kw) == code
 
 
 def test_decode_workspace_sizes(lib):
-    # one split needs no workspace; s splits hold fp32 partial outputs and lse per query row
-    assert lib.attn_decode_workspace_bytes(8, 32, 8, 1, 32768, 128, 1) == 0
-    rows = 8 * 32 * 1
-    got = lib.attn_decode_workspace_bytes(8, 32, 8, 1, 32768, 128, 4)
-    need = 4 * rows * 128 * 4 + 4 * rows * 4
-    assert need <= got <= need + 2 * 256
-    # a requested split count is capped at the number of 128-key tiles
+    # U + P - 1 slots of fp32 partial outputs (R x 128) and lse (R), two int32 per unit, the tile count
+    B, Hq, Hkv, Nq, Nk, P = 8, 32, 8, 1, 32768, 148
+    U, R = B * Hkv, (Hq // Hkv) * Nq
+    slots = U + P - 1
+    need = slots * R * 128 * 4 + slots * R * 4 + 2 * U * 4 + 8
+    got = lib.attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, 128, P)
+    assert need <= got <= need + 5 * 256
+    # the CTA count is capped at the number of key tiles of the largest problem (here 2)
     assert lib.attn_decode_workspace_bytes(1, 2, 2, 1, 256, 128, 50) == \
-        lib.attn_decode_workspace_bytes(1, 2, 2, 1, 256, 128, 2)
+        lib.attn_decode_workspace_bytes(1, 2, 2, 1, 256, 128, 4)
     assert lib.attn_decode_workspace_bytes(1, 2, 2, 1, 256, 64, 2) == 0  # d = 64 unsupported

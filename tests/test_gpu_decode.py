@@ -74,7 +74,7 @@ def check(o, l, O, L, seen, what, heads=None):
         assert np.isneginf(l[~seen]).all(), f"{what}: rows without keys must have lse = -inf"
 
 
-def run(ta, q, k, v, lens, causal, splits, nan_tail=True):
+def run(ta, q, k, v, lens, causal, ctas, nan_tail=True):
     """Call attn_decode on copies of the inputs whose cache entries past kv_lens are NaN."""
     kc, vc = k, v
     if nan_tail and lens is not None:
@@ -83,7 +83,7 @@ def run(ta, q, k, v, lens, causal, splits, nan_tail=True):
             kc[b, :, n:] = float("nan")
             vc[b, :, n:] = float("nan")
     o, l = ta.attn_decode(q.cuda(), kc.cuda(), vc.cuda(), None if lens is None else lens.cuda(), causal=causal,
-                          num_splits=splits)
+                          num_ctas=ctas)
     torch.cuda.synchronize()
     assert ta.attn_check_status() == 0
     return _np(o), l.cpu().numpy().astype(np.float64)
@@ -95,15 +95,17 @@ def _inputs(B, Hq, Hkv, Nq, Nk, dtype, kind, seed, lens):
     return q, k, v, (None if lens is None else torch.tensor(lens, dtype=torch.int32))
 
 
-# (B, Hq, Hkv, Nq, Nk, causal, kv_lens, num_splits, dtype, kind)
+# (B, Hq, Hkv, Nq, Nk, causal, kv_lens, num_ctas, dtype, kind)
 CASES = [
     (2, 8, 8, 1, 300, False, [300, 1], 1, "bf16", "normal"),            # MHA, one row per kv head
-    (2, 32, 8, 1, 1000, False, [1000, 513], 0, "bf16", "k_offset"),      # GQA 4:1, automatic splits
+    (2, 32, 8, 1, 1000, False, [1000, 513], 0, "bf16", "k_offset"),      # GQA 4:1, one CTA per SM
     (1, 32, 8, 4, 777, True, [777], 3, "fp16", "normal"),                 # 16 rows, causal drafts
     (3, 16, 2, 4, 2048, True, [2048, 129, 3], 5, "bf16", "normal"),       # 32 rows; len 3 < Nq
     (2, 8, 1, 8, 640, True, [640, 200], 2, "bf16", "k_offset"),           # 64 rows (MQA)
     (1, 4, 4, 16, 256, False, [0], 1, "bf16", "normal"),                  # empty cache
-    (2, 4, 1, 16, 4096, True, [4096, 4000], 7, "fp16", "normal"),         # 64 rows, 7 splits
+    (2, 4, 1, 16, 4096, True, [4096, 4000], 7, "fp16", "normal"),         # 64 rows, 7 CTAs
+    (5, 8, 2, 1, 900, False, [0, 900, 1, 0, 129], 3, "bf16", "normal"),   # empty units between pieces
+    (6, 8, 8, 1, 256, False, [256, 3, 128, 129, 0, 200], 0, "bf16", "normal"),  # more CTAs than tiles
     (1, 2, 2, 1, 128 * 40, False, None, 1, "bf16", "k_offset"),           # 40 tiles in one CTA
     (2, 24, 8, 2, 3000, True, [3000, 2999], 0, "bf16", "normal"),         # 6 rows, padded to 16
 ]
@@ -111,23 +113,23 @@ CASES = [
 
 @pytest.mark.parametrize("case", CASES)
 def test_decode_small(ta, case):
-    B, Hq, Hkv, Nq, Nk, causal, lens, splits, dtype, kind = case
+    B, Hq, Hkv, Nq, Nk, causal, lens, ctas, dtype, kind = case
     q, k, v, lt = _inputs(B, Hq, Hkv, Nq, Nk, dtype, kind, 90000 + CASES.index(case) * 10, lens)
     ll = lt.tolist() if lt is not None else [Nk] * B
     O, L, seen = expected(q, k, v, ll, causal, 128 ** -0.5)
-    o, l = run(ta, q, k, v, lt, causal, splits)
+    o, l = run(ta, q, k, v, lt, causal, ctas)
     check(o, l, O, L, seen, f"case {case}")
 
 
-def test_split_counts_agree(ta):
-    """1, 2, 5 and 16 splits of the same problem: each within the bars of the oracle, and the lse of
-    the merged splits equal to the single-split lse up to float rounding."""
-    q, k, v, lt = _inputs(2, 32, 8, 2, 5000, "bf16", "normal", 91000, [5000, 4321])
-    O, L, seen = expected(q, k, v, [5000, 4321], True, 128 ** -0.5)
+def test_cta_counts_agree(ta):
+    """1, 2, 5, 16, 37 and 148 CTAs (different cuts of the tile sequence into pieces): each within
+    the bars of the oracle, and the merged lse equal to the one-CTA lse up to float rounding."""
+    q, k, v, lt = _inputs(3, 32, 8, 2, 5000, "bf16", "normal", 91000, [5000, 4321, 77])
+    O, L, seen = expected(q, k, v, [5000, 4321, 77], True, 128 ** -0.5)
     ref = None
-    for s in (1, 2, 5, 16):
+    for s in (1, 2, 5, 16, 37, 148):
         o, l = run(ta, q, k, v, lt, True, s)
-        check(o, l, O, L, seen, f"{s} splits")
+        check(o, l, O, L, seen, f"{s} CTAs")
         if ref is None:
             ref = l
         else:
@@ -174,7 +176,7 @@ def test_unsupported_shapes_raise(ta):
 @pytest.mark.parametrize("cfg", sorted(DECODE_WORKLOADS))
 def test_decode_workloads_full_size(ta, cfg):
     """The named decode workloads at full size, in the launch configuration the benchmark times
-    (automatic splits), checked on 24 sampled (batch, query head) pairs."""
+    (one CTA per SM), checked on 24 sampled (batch, query head) pairs."""
     w = DECODE_WORKLOADS[cfg]
     q, k, v, lt = make_decode_inputs(w)
     rng = np.random.default_rng(cfg)

@@ -143,11 +143,11 @@ def attn_fwd(q, k, v, causal=False, scale=None, mode="bf16_exact", out=None, lse
     return o, l
 
 
-def attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits=0) -> int:
-    return int(load_library().attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits))
+def attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_ctas=0) -> int:
+    return int(load_library().attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_ctas))
 
 
-def attn_decode(q, k_cache, v_cache, kv_lens=None, causal=False, scale=None, num_splits=0, out=None, lse=True,
+def attn_decode(q, k_cache, v_cache, kv_lens=None, causal=False, scale=None, num_ctas=0, out=None, lse=True,
                 workspace=None, stream=None):
     """Attention of q [B, Hq, Nq, d] against the first kv_lens[b] keys of k_cache / v_cache
     [B, Hkv, Nk, d] (kv_lens: int32 CUDA tensor [B] or None for all Nk).  Returns (o, lse or None)."""
@@ -169,11 +169,11 @@ def attn_decode(q, k_cache, v_cache, kv_lens=None, causal=False, scale=None, num
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty_like(q) if out is None else out
     l = _lse_arg(lse, (B, Hq, Nq), q.device)
-    ws_bytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits)
+    ws_bytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_ctas)
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
     rc = lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kv_lens), _ptr(o), _ptr(l), B, Hq, Hkv, Nq,
-                         Nk, d, int(bool(causal)), scale, DTYPES[q.dtype], int(num_splits), _ptr(workspace),
+                         Nk, d, int(bool(causal)), scale, DTYPES[q.dtype], int(num_ctas), _ptr(workspace),
                          0 if workspace is None else workspace.numel() * workspace.element_size(),
                          _stream(stream))
     _check(rc, "attn_decode")

@@ -411,49 +411,45 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   return ATTN_OK;
 }
 
-size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {
-  if (check_decode_shape(B, Hq, Hkv, Nq, Nk, d, num_splits)) return 0;
-  return decode_ws(B, Hq, Nq, decode_splits(B, Hkv, Nk, num_splits)).total;
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas) {
+  if (check_decode_shape(B, Hq, Hkv, Nq, Nk, d, num_ctas)) return 0;
+  return decode_ws(B, Hkv, (Hq / Hkv) * Nq, decode_ctas(B, Hkv, Nk, num_ctas)).total;
 }
 
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens, void* o, float* lse,
-                int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale, int dtype, int num_splits,
+                int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale, int dtype, int num_ctas,
                 void* workspace, size_t ws_bytes, void* stream) {
   if (!q || !k_cache || !v_cache || !o) return ATTN_ERR_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_ARG;
   if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_ARG;
-  int rc = check_decode_shape(B, Hq, Hkv, Nq, Nk, d, num_splits);
+  int rc = check_decode_shape(B, Hq, Hkv, Nq, Nk, d, num_ctas);
   if (rc) return rc;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || (lse && !aligned16(lse)) ||
       (reinterpret_cast<uintptr_t>(kv_lens) & 3u))
     return ATTN_ERR_ALIGN;
-  const int nsplit = decode_splits(B, Hkv, Nk, num_splits);
-  if ((long long)B * Hkv * nsplit > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;  // grid x extent
-  const DecWs w = decode_ws(B, Hq, Nq, nsplit);
-  if (w.total > 0) {
-    if (!workspace || ws_bytes < w.total) return ATTN_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
-  }
+  const int R = (Hq / Hkv) * Nq;
+  const int ctas = decode_ctas(B, Hkv, Nk, num_ctas);
+  const DecWs w = decode_ws(B, Hkv, R, ctas);
+  if (!workspace || ws_bytes < w.total) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
   DecParams p{};
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.Nq = Nq;
   p.Nk = Nk;
-  p.R = (Hq / Hkv) * Nq;
+  p.R = R;
   p.causal = causal;
-  p.nsplit = nsplit;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.kv_lens = kv_lens;
-  p.o = o;
-  p.lse = lse;
-  if (w.total > 0) {
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    p.part_o = reinterpret_cast<float*>(ws + w.part_o);
-    p.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
-  }
-  return launch_decode(q, k_cache, v_cache, dtype, p, static_cast<cudaStream_t>(stream));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.part_o = reinterpret_cast<float*>(ws + w.part_o);
+  p.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
+  p.unit_first = reinterpret_cast<int*>(ws + w.unit_first);
+  p.unit_count = reinterpret_cast<int*>(ws + w.unit_count);
+  p.total = reinterpret_cast<long long*>(ws + w.tiles);
+  return launch_decode(q, k_cache, v_cache, o, lse, dtype, ctas, p, static_cast<cudaStream_t>(stream));
 }
 
 int attn_check_status(void) {

@@ -47,45 +47,54 @@ struct DecParams {
   int B, Hq, Hkv, Nq, Nk;
   int R;                 // (Hq / Hkv) * Nq query rows per kv head
   int causal;
-  int nsplit;            // CTAs per (batch, kv head)
   float scale_log2;      // scale * log2(e)
   const int* kv_lens;    // [B] cached keys per sequence (clamped to [0, Nk]); null: all Nk
-  void* o;               // nsplit == 1: [B, Hq, Nq, 128] 16-bit
-  float* lse;            // nsplit == 1: [B, Hq, Nq] or null
-  float* part_o;         // nsplit > 1: [nsplit, B*Hq*Nq, 128] fp32, normalised per split
-  float* part_lse;       // nsplit > 1: [nsplit, B*Hq*Nq]
+  // Partial results of the pieces (see the scheduling note in attn_decode_kernel): the piece of
+  // unit u processed by CTA i goes to slot u + i, so U + P - 1 slots cover every partition.
+  float* part_o;         // [slots, R, 128] fp32, normalised per piece
+  float* part_lse;       // [slots, R]
+  int* unit_first;       // [U] the CTA holding each unit's first tile
+  int* unit_count;       // [U] CTAs from there to the one holding its last tile (some may be empty)
+  long long* total;      // [1] key tiles in all (written by CTA 0)
 };
 
 template <int RP>
 struct DecCfg {
   static constexpr int D = 128;
-  static constexpr int CW = RP < 32 ? RP : 32;   // query columns per softmax thread
-  static constexpr int NWG = RP / CW;            // softmax warpgroups
+  // Query columns per softmax thread: two warpgroups share every tile (each takes half of the
+  // columns), so every SM sub-partition runs two softmax warps.
+#ifndef TATTN_DEC_WG
+#define TATTN_DEC_WG 2
+#endif
+  static constexpr int NWG_WANT = TATTN_DEC_WG < RP / 8 ? TATTN_DEC_WG : RP / 8;  // at least 8 columns
+  static constexpr int NWG = RP / 32 > NWG_WANT ? RP / 32 : NWG_WANT;          // at most 32 columns
+  static constexpr int CW = RP / NWG;
   static constexpr int kSoftmaxWarps = 4 * NWG;
   static constexpr int kTmaWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
   static constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
   static constexpr int PANEL = 128 * 128;        // 128 keys x 64 channels x 2 B (one TMA box)
   static constexpr int KV_TILE = 2 * PANEL;
-  static constexpr int Q_PANEL = RP * 128, Q_TILE = 2 * Q_PANEL;
+  static constexpr int Q_PANEL = RP * 128, Q_TILE = 2 * Q_PANEL;  // two Q buffers (pieces alternate)
   static constexpr int P_PANEL = RP * 128, P_TILE = 2 * P_PANEL;  // RP rows x 64 keys x 2 B per panel
-  static constexpr int KS = 3;
-  static constexpr int VS = RP <= 32 ? 3 : 2;
+  static constexpr int KS = RP <= 32 ? 3 : 2;
+  static constexpr int VS = RP <= 16 ? 3 : 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_P = OFF_Q + Q_TILE;
+  static constexpr int OFF_P = OFF_Q + 2 * Q_TILE;
   static constexpr int OFF_K = OFF_P + 2 * P_TILE;
   static constexpr int OFF_V = OFF_K + KS * KV_TILE;
   static constexpr int OFF_RED = OFF_V + VS * KV_TILE;    // float [2][4][RP]: per-warp column maxima
   static constexpr int OFF_LRED = OFF_RED + 2 * RP * 16;  // float [RP][4]: per-warp row sums
   static constexpr int OFF_M = OFF_LRED + RP * 16;        // float [2][RP]: running column maxima
-  static constexpr int OFF_BAR = OFF_M + 2 * RP * 4;
-  // q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2], o_done,
-  // o_final, drain
-  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 4 + 3;
+  static constexpr int OFF_SCHED = OFF_M + 2 * RP * 4;    // long long [8]: this CTA's tile range
+  static constexpr int OFF_BAR = OFF_SCHED + 64;
+  // q_full[2], q_empty[2], k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], s_free[2],
+  // p_full[2], o_done[2], o_final[2], o_free[2], drain
+  static constexpr int NBAR = 4 + 2 * KS + 2 * VS + 12 + 1;
   static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
   static constexpr int SMEM_BYTES = SMEM_USED + 1024;
-  static constexpr uint32_t TMEM_COLS = 3 * RP <= 64 ? 64u : (3 * RP <= 128 ? 128u : 256u);
+  static constexpr uint32_t TMEM_COLS = 4 * RP <= 64 ? 64u : (4 * RP <= 128 ? 128u : 256u);
   __host__ __device__ static constexpr uint32_t tm_s(int buf) { return (uint32_t)(buf * RP); }
-  static constexpr uint32_t TM_O = 2 * RP;
+  __host__ __device__ static constexpr uint32_t tm_o(int buf) { return (uint32_t)((2 + buf) * RP); }
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(RP % 16 == 0 && RP <= 64, "N of the M = 128 MMAs");
 };
@@ -128,7 +137,10 @@ __device__ __forceinline__ uint16_t to16(float x) {
 
 template <int CW>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CW]) {
-  if constexpr (CW == 16) {
+  if constexpr (CW == 8) {
+    tmem_ld8(taddr, r);
+    tmem_ld_wait8(r);
+  } else if constexpr (CW == 16) {
     tmem_ld16(taddr, r);
     tmem_ld_wait16(r);
   } else {
@@ -138,8 +150,123 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CW]) 
 }
 template <int CW>
 __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[CW]) {
-  if constexpr (CW == 16) tmem_st16(taddr, r);
+  if constexpr (CW == 8) tmem_st8(taddr, r);
+  else if constexpr (CW == 16) tmem_st16(taddr, r);
   else tmem_st32(taddr, r);
+}
+
+__device__ __forceinline__ int dec_len(const DecParams& p, int b) {
+  const int len = p.kv_lens ? __ldg(&p.kv_lens[b]) : p.Nk;
+  return min(max(len, 0), p.Nk);
+}
+
+// Walks this CTA's contiguous range [g, g_end) of the global key-tile sequence.  The sequence lists
+// the units (batch b, kv head h) in order, each with ceil(len_b / 128) tiles; the part of the range
+// that falls in one unit is a "piece".  Every role (producer, MMA issuer, softmax) runs its own
+// copy of the cursor and so visits the same tiles in the same order.
+struct DecCursor {
+  int b, h, lt;          // current unit and local tile index in it
+  int ps, pe;            // current piece: local tiles [ps, pe)
+  int ntb, len;          // tiles and keys of batch b
+  int k;                 // pieces started so far (selects the Q and O buffers)
+  int gl;                // tiles visited so far (selects ring stages and S/P buffers)
+  long long g, g_end;    // global index of tile lt; end of the CTA's range
+
+  __device__ __forceinline__ void init(const DecParams& p, const long long* sched) {
+    g = sched[0];
+    g_end = sched[1];
+    b = (int)sched[3];
+    h = (int)sched[4];
+    lt = (int)sched[5];
+    k = 0;
+    gl = 0;
+    if (g < g_end) {
+      len = dec_len(p, b);
+      ntb = (len + 127) / 128;
+      ps = lt;
+      pe = (int)min((long long)ntb, (long long)lt + (g_end - g));
+    }
+  }
+  __device__ __forceinline__ bool valid() const { return g < g_end; }
+  __device__ __forceinline__ bool first() const { return lt == ps; }
+  __device__ __forceinline__ bool last() const { return lt + 1 == pe; }
+  __device__ __forceinline__ int unit(const DecParams& p) const { return b * p.Hkv + h; }
+  __device__ __forceinline__ void next(const DecParams& p) {
+    ++lt;
+    ++g;
+    ++gl;
+    if (lt < pe || g >= g_end) return;
+    ++k;  // next piece: the next unit that has tiles
+    if (++h == p.Hkv) {
+      h = 0;
+      do {
+        if (++b >= p.B) {  // (only if kv_lens changed during the call)
+          g = g_end;
+          return;
+        }
+        len = dec_len(p, b);
+        ntb = (len + 127) / 128;
+      } while (ntb == 0);
+    }
+    lt = 0;
+    ps = 0;
+    pe = (int)min((long long)ntb, g_end - g);
+  }
+};
+
+// The CTA's share of the key tiles: with T tiles in all and P CTAs, CTA i takes
+// [floor(i T / P), floor((i + 1) T / P)).  One warp scans kv_lens twice (total, then the unit that
+// holds the first tile).  sched = {first, end, T, b, h, local tile}.
+__device__ void dec_schedule(const DecParams& p, long long* sched, int lane) {
+  const unsigned FULL = 0xffffffffu;
+  long long total = 0;
+  for (int base = 0; base < p.B; base += 32) {
+    const int bb = base + lane;
+    long long n = bb < p.B ? (long long)((dec_len(p, bb) + 127) / 128) * p.Hkv : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(FULL, n, o);
+      if (lane >= o) n += y;
+    }
+    total += __shfl_sync(FULL, n, 31);
+  }
+  const long long P = gridDim.x, i = blockIdx.x;
+  const long long g0 = total * i / P, g1 = total * (i + 1) / P;
+  int fb = 0, fh = 0, flt = 0;
+  if (g0 < g1) {
+    long long run = 0;
+    for (int base = 0; base < p.B; base += 32) {
+      const int bb = base + lane;
+      const int ntb = bb < p.B ? (dec_len(p, bb) + 127) / 128 : 0;
+      const long long n = (long long)ntb * p.Hkv;
+      long long incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(FULL, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const long long excl = run + incl - n;
+      const unsigned hit = __ballot_sync(FULL, n > 0 && g0 >= excl && g0 < excl + n);
+      if (hit) {
+        const int src = __ffs(hit) - 1;
+        const long long off = __shfl_sync(FULL, g0 - excl, src);
+        const int nt_src = __shfl_sync(FULL, ntb, src);
+        fb = base + src;
+        fh = (int)(off / nt_src);
+        flt = (int)(off % nt_src);
+        break;
+      }
+      run += __shfl_sync(FULL, incl, 31);
+    }
+  }
+  if (lane == 0) {
+    sched[0] = g0;
+    sched[1] = g1;
+    sched[2] = total;
+    sched[3] = fb;
+    sched[4] = fh;
+    sched[5] = flt;
+  }
 }
 
 template <int RP, bool FP16>
@@ -152,15 +279,18 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars;
-  uint64_t* k_full = q_full + 1;
+  uint64_t* q_empty = q_full + 2;
+  uint64_t* k_full = q_empty + 2;
   uint64_t* k_empty = k_full + C::KS;
   uint64_t* v_full = k_empty + C::KS;
   uint64_t* v_empty = v_full + C::VS;
   uint64_t* s_full = v_empty + C::VS;
-  uint64_t* p_full = s_full + 2;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
   uint64_t* o_done = p_full + 2;
-  uint64_t* o_final = o_done + 1;
-  uint64_t* drain = o_final + 1;
+  uint64_t* o_final = o_done + 2;
+  uint64_t* o_free = o_final + 2;
+  uint64_t* drain = o_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* sQ = smem + C::OFF_Q;
@@ -170,15 +300,22 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
   float* lred = reinterpret_cast<float*>(smem + C::OFF_LRED);
   float* m_sh = reinterpret_cast<float*>(smem + C::OFF_M);
+  long long* sched = reinterpret_cast<long long*>(smem + C::OFF_SCHED);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], C::kSoftmaxWarps);
+      mbar_init(&p_full[i], C::kSoftmaxWarps);
+      mbar_init(&o_done[i], 1);
+      mbar_init(&o_final[i], 1);
+      mbar_init(&o_free[i], C::kSoftmaxWarps);
+    }
     for (int i = 0; i < C::KS; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < C::VS; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], C::kSoftmaxWarps); }
-    mbar_init(o_done, 1);
-    mbar_init(o_final, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -187,52 +324,57 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == C::kTmaWarp && lane == 0) {
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
+  if (warp == C::kTmaWarp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
+    dec_schedule(p, sched, lane);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  // ---- work item: (batch, kv head) x split of that sequence's key tiles ----
-  const int bkv = (int)(blockIdx.x / (unsigned)p.nsplit);
-  const int split = (int)blockIdx.x - bkv * p.nsplit;
-  const int b = bkv / p.Hkv;
-  int len = p.kv_lens ? __ldg(&p.kv_lens[b]) : p.Nk;
-  len = min(max(len, 0), p.Nk);
-  const int ntiles = (len + 127) / 128;
-  const int chunk = (ntiles + p.nsplit - 1) / p.nsplit;
-  const int t_lo = min(split * chunk, ntiles);
-  const int nt = min(t_lo + chunk, ntiles) - t_lo;
+  const long long total_tiles = sched[2];
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.total = total_tiles;
 
   if (warp == C::kTmaWarp) {
     // ================================ TMA producer ================================
-    if (lane == 0 && nt > 0) {
+    if (lane == 0) {
       const uint64_t pol = policy_evict_first();  // every cached byte is read once
-      int k_issued = 0, v_issued = 0;
+      DecCursor c;
+      c.init(p, sched);
+      int q_issued = 0, k_issued = 0, v_issued = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, C::Q_TILE);
-      for (int pn = 0; pn < 2; ++pn) tma_load_3d(sQ + pn * C::Q_PANEL, &tmQ, pn * 64, 0, bkv, q_full, pol);
-      for (int j = 0; j < nt && ok; ++j) {
-        const int ks = j % C::KS, vs = j % C::VS;
-        const int key0 = (t_lo + j) * 128;
-        if (!(ok = mbar_wait(&k_empty[ks], ((j / C::KS) & 1) ^ 1, abort_flag, WD_LOAD + 1))) break;
+      while (c.valid()) {
+        const int u = c.unit(p);
+        if (c.first()) {  // a new piece: the unit's query rows
+          const int qb = c.k & 1;
+          if (!(ok = mbar_wait(&q_empty[qb], ((c.k >> 1) & 1) ^ 1, abort_flag, WD_LOAD + 0))) break;
+          mbar_arrive_expect_tx(&q_full[qb], C::Q_TILE);
+          for (int pn = 0; pn < 2; ++pn)
+            tma_load_3d(sQ + qb * C::Q_TILE + pn * C::Q_PANEL, &tmQ, pn * 64, 0, u, &q_full[qb], pol);
+          q_issued = c.k + 1;
+        }
+        const int ks = c.gl % C::KS, vs = c.gl % C::VS;
+        const int key0 = c.lt * 128;
+        if (!(ok = mbar_wait(&k_empty[ks], ((c.gl / C::KS) & 1) ^ 1, abort_flag, WD_LOAD + 1))) break;
         mbar_arrive_expect_tx(&k_full[ks], C::KV_TILE);
         for (int pn = 0; pn < 2; ++pn)
-          tma_load_3d(sK + ks * C::KV_TILE + pn * C::PANEL, &tmK, pn * 64, key0, bkv, &k_full[ks], pol);
-        k_issued = j + 1;
-        if (!(ok = mbar_wait(&v_empty[vs], ((j / C::VS) & 1) ^ 1, abort_flag, WD_LOAD + 2))) break;
+          tma_load_3d(sK + ks * C::KV_TILE + pn * C::PANEL, &tmK, pn * 64, key0, u, &k_full[ks], pol);
+        k_issued = c.gl + 1;
+        if (!(ok = mbar_wait(&v_empty[vs], ((c.gl / C::VS) & 1) ^ 1, abort_flag, WD_LOAD + 2))) break;
         mbar_arrive_expect_tx(&v_full[vs], C::KV_TILE);
         for (int pn = 0; pn < 2; ++pn)
-          tma_load_3d(sV + vs * C::KV_TILE + pn * C::PANEL, &tmV, pn * 64, key0, bkv, &v_full[vs], pol);
-        v_issued = j + 1;
+          tma_load_3d(sV + vs * C::KV_TILE + pn * C::PANEL, &tmV, pn * 64, key0, u, &v_full[vs], pol);
+        v_issued = c.gl + 1;
+        c.next(p);
       }
       if (!ok) {
         // every issued copy must land before the CTA's shared memory is released
-        mbar_wait(q_full, 0, nullptr, WD_DRAIN + 1, 200000000ull);
+        for (int j = max(0, q_issued - 2); j < q_issued; ++j)
+          mbar_wait(&q_full[j & 1], (j >> 1) & 1, nullptr, WD_DRAIN + 1, 200000000ull);
         for (int j = max(0, k_issued - C::KS); j < k_issued; ++j)
           mbar_wait(&k_full[j % C::KS], (j / C::KS) & 1, nullptr, WD_DRAIN + 2, 200000000ull);
         for (int j = max(0, v_issued - C::VS); j < v_issued; ++j)
@@ -242,33 +384,60 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
     __syncwarp();
   } else if (warp == C::kMmaWarp) {
     // ================================ MMA issuer ================================
-    if (lane == 0 && nt > 0) {
+    // Two in-order streams of tcgen05 work, issued by one thread as their inputs become ready:
+    //   S^T(h) = K(h) Q^T   needs K(h), the piece's Q, and S^T buffer h % 2 read out (S^T(h - 2)),
+    //   O^T += V^T P^T(g)   needs P^T(g), V(g) and, for a piece's first tile, its O buffer free.
+    // Polling both with non-blocking tests keeps either stream from stalling behind the other
+    // (S^T two tiles ahead often waits for its K tile while P^T is already there).
+    if (lane == 0) {
       const uint32_t q_addr = smem_u32(sQ), p_addr = smem_u32(sP), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      bool ok = mbar_wait(q_full, 0, abort_flag, WD_MMA + 1);
-      // S^T of tiles 0 and 1 up front; S^T(j + 2) is issued right after O^T += V^T P^T(j)
-      for (int j = 0; j < 2 && j < nt && ok; ++j) {
-        if (!(ok = mbar_wait(&k_full[j % C::KS], (j / C::KS) & 1, abort_flag, WD_MMA + 2))) break;
-        tc_fence_after();
-        issue_kq<RP, FP16>(tmem + C::tm_s(j), k_addr + (j % C::KS) * C::KV_TILE, q_addr);
-        mma_commit(&s_full[j]);
-        mma_commit(&k_empty[j % C::KS]);
-      }
-      for (int j = 0; j < nt && ok; ++j) {
-        const int vs = j % C::VS;
-        if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, WD_MMA + 3))) break;
-        if (!(ok = mbar_wait(&v_full[vs], (j / C::VS) & 1, abort_flag, WD_MMA + 4))) break;
-        tc_fence_after();
-        issue_vp<RP, FP16>(tmem + C::TM_O, v_addr + vs * C::KV_TILE, p_addr + (j & 1) * C::P_TILE, j > 0);
-        mma_commit(&v_empty[vs]);
-        mma_commit(o_done);  // one phase per tile
-        if (j + 1 == nt) mma_commit(o_final);
-        if (j + 2 < nt) {
-          const int ks = (j + 2) % C::KS;
-          if (!(ok = mbar_wait(&k_full[ks], ((j + 2) / C::KS) & 1, abort_flag, WD_MMA + 5))) break;
-          tc_fence_after();
-          issue_kq<RP, FP16>(tmem + C::tm_s(j & 1), k_addr + ks * C::KV_TILE, q_addr);
-          mma_commit(&s_full[j & 1]);
-          mma_commit(&k_empty[ks]);
+      DecCursor cs, cp;
+      cs.init(p, sched);
+      cp.init(p, sched);
+      bool ok = true;
+      unsigned long long t_idle = 0;
+      uint32_t spins = 0;
+      while (cp.valid()) {
+        bool did = false;
+        if (cs.valid()) {
+          const int h = cs.gl, qb = cs.k & 1, ks = h % C::KS;
+          if ((h < 2 || mbar_test(&s_free[h & 1], ((h - 2) >> 1) & 1)) &&
+              (!cs.first() || mbar_test(&q_full[qb], (cs.k >> 1) & 1)) && mbar_test(&k_full[ks], (h / C::KS) & 1)) {
+            tc_fence_after();
+            issue_kq<RP, FP16>(tmem + C::tm_s(h & 1), k_addr + ks * C::KV_TILE, q_addr + qb * C::Q_TILE);
+            mma_commit(&s_full[h & 1]);
+            mma_commit(&k_empty[ks]);
+            if (cs.last()) mma_commit(&q_empty[qb]);
+            cs.next(p);
+            did = true;
+          }
+        }
+        {
+          const int g = cp.gl, vs = g % C::VS, ob = cp.k & 1;
+          if (cp.gl < cs.gl && mbar_test(&p_full[g & 1], (g >> 1) & 1) && mbar_test(&v_full[vs], (g / C::VS) & 1) &&
+              (!cp.first() || mbar_test(&o_free[ob], ((cp.k >> 1) & 1) ^ 1))) {
+            tc_fence_after();
+            issue_vp<RP, FP16>(tmem + C::tm_o(ob), v_addr + vs * C::KV_TILE, p_addr + (g & 1) * C::P_TILE,
+                               !cp.first());
+            mma_commit(&v_empty[vs]);
+            mma_commit(&o_done[g & 1]);  // one phase per two tiles
+            if (cp.last()) mma_commit(&o_final[ob]);
+            cp.next(p);
+            did = true;
+          }
+        }
+        // bounded: no progress for kWaitTimeoutNs (or another role's abort) ends the loop
+        if (did) {
+          spins = 0;
+        } else if ((++spins & 63u) == 0u) {
+          if (*abort_flag) { ok = false; break; }
+          const unsigned long long now = globaltimer_ns();
+          if (spins == 64u) t_idle = now;
+          else if (now - t_idle > kWaitTimeoutNs) {
+            report_timeout(abort_flag, WD_MMA + 7);
+            ok = false;
+            break;
+          }
         }
       }
       if (!ok) {
@@ -285,31 +454,39 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
     const int c0 = wg * CW;          // first query column of this warpgroup
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int bar_id = 1 + wg;
-    const int rows_total = p.B * p.Hkv * p.R;
-    // Keys [0, lim(c)) are visible to query column c: lim = len, or under the causal mask
-    // len - Nq + 1 + (c mod Nq).  Tiles that end at or before `edge` need no mask at all.  Padded
-    // columns (c >= R) are never masked: their Q rows are zeros, they only ever feed their own
-    // columns of O^T and l, and nothing of them is written out.
-    const int causal_base = len - p.Nq + 1;
-    const int edge = p.causal ? min(len, causal_base) : len;
     // P^T store address of element (row c, key t): two 64-key panels, 128-byte swizzle
     const uint32_t p_base = smem_u32(sP) + (uint32_t)(t >> 6) * C::P_PANEL + (uint32_t)(t & 7) * 2;
     const uint32_t p_chunk = (uint32_t)((t & 63) >> 3);
     float l_run[CW];
-#pragma unroll
-    for (int r = 0; r < CW; ++r) l_run[r] = 0.f;
     bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      const int buf = j & 1;
-      bool okw = mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, WD_SOFTMAX + 1);
+    DecCursor cur;
+    cur.init(p, sched);
+    while (cur.valid()) {
+      const int g = cur.gl, buf = g & 1;
+      const bool first = cur.first();
+      if (first) {
+#pragma unroll
+        for (int r = 0; r < CW; ++r) l_run[r] = 0.f;
+      }
+      const int len = cur.len;
+      // Keys [0, lim(c)) are visible to query column c: lim = len, or under the causal mask
+      // len - Nq + 1 + (c mod Nq).  Tiles that end at or before `edge` need no mask at all.
+      // Padded columns (c >= R) are never masked: their Q rows are zeros, they only ever feed
+      // their own columns of O^T and l, and nothing of them is written out.
+      const int causal_base = len - p.Nq + 1;
+      const int edge = p.causal ? min(len, causal_base) : len;
+      bool okw = mbar_wait(&s_full[buf], (g >> 1) & 1, abort_flag, WD_SOFTMAX + 1);
       okw = __all_sync(0xffffffffu, okw);
       float s[CW];
-      const int tile0 = (t_lo + j) * 128;
+      const int tile0 = cur.lt * 128;
       const int key = tile0 + t;
       if (okw) {
         tc_fence_after();
         uint32_t raw[CW];
         tmem_ld_cols<CW>(tmem + C::tm_s(buf) + (uint32_t)c0 + lane_off, raw);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[buf]);  // the MMA issuer may overwrite S^T(buf) now
 #pragma unroll
         for (int r = 0; r < CW; ++r) s[r] = __uint_as_float(raw[r]);
         if (tile0 + 128 > edge) {  // (the same for the whole warpgroup)
@@ -337,9 +514,16 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
       }
       if (!(ok = named_bar_and(bar_id, 128, okw && ok))) break;
       // Column maxima over the 128 keys and the lazy update of the running max m (kept in shared
-      // memory, double-buffered by tile parity: every thread computes the same m, lane r of the
-      // group's first warp stores column c0 + r).  Then P^T(j) = exp2(s * scale_log2 - m), with
-      // masked keys giving exp2(-inf) = 0, and the per-key partial row sums.
+      // memory, double-buffered by tile parity: every thread computes the same m, one thread
+      // stores it).  Then P^T = exp2(s * scale_log2 - m), with masked keys giving exp2(-inf) = 0,
+      // and the per-key partial row sums.
+      // P^T(buf) was read by P V of tile g - 2: wait for phase (g - 2) / 2 of o_done[buf].  Every
+      // tile waits for the next phase of one of the two barriers in turn, and P V of tile g needs
+      // this tile's P^T, so the awaited phase is always the current or the last completed one.
+      if (g >= 2) {
+        bool okp = mbar_wait(&o_done[buf], ((g - 2) >> 1) & 1, abort_flag, WD_SOFTMAX + 5);
+        ok = __all_sync(0xffffffffu, okp) && ok;
+      }
       float alpha[CW];
       bool resc = false;
       const uint32_t pb = p_base + (uint32_t)buf * C::P_TILE;
@@ -349,7 +533,7 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
 #pragma unroll
       for (int q4 = 0; q4 < CW / 4; ++q4) {  // four columns at a time: vector loads of the maxima
         const float4 a = rd[q4], b4 = rd[RP / 4 + q4], c4 = rd[2 * (RP / 4) + q4], d4 = rd[3 * (RP / 4) + q4];
-        const float4 m4 = j > 0 ? mo[q4] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        const float4 m4 = first ? make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY) : mo[q4];
         const float wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b4.x, b4.y, b4.z, b4.w};
         const float wc[4] = {c4.x, c4.y, c4.z, c4.w}, wd[4] = {d4.x, d4.y, d4.z, d4.w};
         const float mold[4] = {m4.x, m4.y, m4.z, m4.w};
@@ -376,28 +560,29 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
           st_shared_u16(pb + (uint32_t)c * 128 + ((p_chunk ^ (uint32_t)(c & 7)) << 4), to16<FP16>(pv));
         }
       }
-      // (resc and j are the same for every thread of the warpgroup)
-      if (resc && j > 0) {
-        // O^T must hold P V of tile j - 1 before it is rescaled.  The waiter is never more than
-        // one phase behind: S^T(j) was issued after P V of tile j - 2, and P V of tile j waits
-        // for this warpgroup's P^T(j).
-        bool oko = mbar_wait(o_done, (j - 1) & 1, abort_flag, WD_SOFTMAX + 2);
+      // (resc and first are the same for every thread of the warpgroup)
+      if (resc && !first) {
+        // O^T must hold P V of the previous tile before it is rescaled: phase (g - 1) / 2 of
+        // o_done[(g - 1) & 1] (the previous tile awaited its phase before, and P V of tile g + 1
+        // waits for P^T(g + 1), so no later phase of that barrier can be done).
+        bool oko = mbar_wait(&o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, WD_SOFTMAX + 2);
         oko = __all_sync(0xffffffffu, oko);
         if (oko) {
           tc_fence_after();
+          const uint32_t to = tmem + C::tm_o(cur.k & 1) + (uint32_t)c0 + lane_off;
           uint32_t o[CW];
-          tmem_ld_cols<CW>(tmem + C::TM_O + (uint32_t)c0 + lane_off, o);
+          tmem_ld_cols<CW>(to, o);
 #pragma unroll
           for (int r = 0; r < CW; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
-          tmem_st_cols<CW>(tmem + C::TM_O + (uint32_t)c0 + lane_off, o);
+          tmem_st_cols<CW>(to, o);
           tmem_st_wait();
         }
         ok = oko;  // on failure the abort flag is raised: the next wait returns at once
       }
       // the sequence's last tile: zero the V rows of keys >= len (never valid cache entries)
       if (wg == 0 && tile0 + 128 > len) {
-        const int vs = j % C::VS;
-        const bool okv = mbar_wait(&v_full[vs], (j / C::VS) & 1, abort_flag, WD_SOFTMAX + 3);
+        const int vs = g % C::VS;
+        const bool okv = mbar_wait(&v_full[vs], (g / C::VS) & 1, abort_flag, WD_SOFTMAX + 3);
         if (okv && key >= len) {
           const uint32_t vrow = smem_u32(sV) + (uint32_t)vs * C::KV_TILE + (uint32_t)t * 128;
 #pragma unroll
@@ -411,47 +596,51 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[buf]);
-    }
 
-    // ---- epilogue: reduce the row sums over the 128 keys, normalise, write ----
-    bool oke = ok;
-    if (nt > 0 && oke) oke = mbar_wait(o_final, 0, abort_flag, WD_SOFTMAX + 4);
+      if (cur.last()) {
+        // ---- end of a piece: reduce the row sums over the 128 keys, normalise, write the
+        // piece's partial output and lse to slot (unit + CTA index) ----
+        const int ob = cur.k & 1;
+        bool oke = ok && mbar_wait(&o_final[ob], (cur.k >> 1) & 1, abort_flag, WD_SOFTMAX + 4);
 #pragma unroll
-    for (int r = 0; r < CW; ++r) {
-      float v = l_run[r];
+        for (int r = 0; r < CW; ++r) {
+          float v = l_run[r];
 #pragma unroll
-      for (int sh = 16; sh > 0; sh >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sh);
-      if (lane == 0) lred[(c0 + r) * 4 + wq] = v;
-    }
-    if (named_bar_and(bar_id, 128, oke)) {
-      uint32_t o[CW];
-      if (nt > 0) {
+          for (int sh = 16; sh > 0; sh >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sh);
+          if (lane == 0) lred[(c0 + r) * 4 + wq] = v;
+        }
+        if (!(ok = named_bar_and(bar_id, 128, oke))) break;
         tc_fence_after();
-        tmem_ld_cols<CW>(tmem + C::TM_O + (uint32_t)c0 + lane_off, o);
-      } else {
+        uint32_t o[CW];
+        tmem_ld_cols<CW>(tmem + C::tm_o(ob) + (uint32_t)c0 + lane_off, o);
+        const int u = cur.unit(p);
+        const long long slot = (long long)u + blockIdx.x;
+        const float* m_last = m_sh + buf * RP;
 #pragma unroll
-        for (int r = 0; r < CW; ++r) o[r] = 0u;
-      }
-      const float* m_last = m_sh + ((nt - 1) & 1) * RP;
-#pragma unroll
-      for (int r = 0; r < CW; ++r) {
-        const int c = c0 + r;
-        if (c < p.R) {
-          const float4 l4 = *reinterpret_cast<const float4*>(&lred[c * 4]);
-          const float lsum = (l4.x + l4.y) + (l4.z + l4.w);
-          const float val = lsum > 0.f ? __uint_as_float(o[r]) / lsum : 0.f;
-          const size_t row = (size_t)bkv * p.R + c;
-          float lse = -INFINITY;
-          if (t == r && lsum > 0.f) lse = (m_last[c] + __log2f(lsum)) * 0.69314718055994531f;
-          if (p.nsplit == 1) {
-            reinterpret_cast<uint16_t*>(p.o)[row * 128 + t] = to16<FP16>(val);
-            if (p.lse != nullptr && t == r) p.lse[row] = lse;
-          } else {
-            p.part_o[((size_t)split * rows_total + row) * 128 + t] = val;
-            if (t == r) p.part_lse[(size_t)split * rows_total + row] = lse;
+        for (int r = 0; r < CW; ++r) {
+          const int c = c0 + r;
+          if (c < p.R) {
+            const float4 l4 = *reinterpret_cast<const float4*>(&lred[c * 4]);
+            const float lsum = (l4.x + l4.y) + (l4.z + l4.w);
+            p.part_o[(slot * p.R + c) * 128 + t] = lsum > 0.f ? __uint_as_float(o[r]) / lsum : 0.f;
+            if (t == r)
+              p.part_lse[slot * p.R + c] =
+                  lsum > 0.f ? (m_last[c] + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
           }
         }
+        if (cur.ps == 0 && threadIdx.x == 0) {
+          // this CTA holds the unit's first tile: record which CTAs hold its pieces.  The unit's
+          // last tile lies in CTA ceil((g_u + n) P / T) - 1, g_u being its first global tile.
+          const long long gu = cur.g - cur.lt, P = gridDim.x;
+          const long long i_last = ((gu + cur.ntb) * P + total_tiles - 1) / total_tiles - 1;
+          p.unit_first[u] = (int)blockIdx.x;
+          p.unit_count[u] = (int)(i_last - blockIdx.x + 1);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[ob]);
       }
+      cur.next(p);
     }
     tmem_st_wait();
   }
@@ -464,26 +653,41 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
   }
 }
 
-// Merge of the splits of one query row: O = sum_s w_s O_s / sum_s w_s with w_s = exp(lse_s - max),
-// lse = max + log(sum_s w_s).  One CTA of 128 threads (one per channel) per row.
+// Merge of the pieces of one query row: O = sum_s w_s O_s / sum_s w_s with w_s = exp(lse_s - max),
+// lse = max + log(sum_s w_s), in one pass with a running max.  One CTA of 128 threads (one per
+// channel) per row; a row whose sequence holds no key gets O = 0 and lse = -inf.  The pieces of
+// unit u are in slots u + i for the CTAs i from unit_first[u] on; when there are fewer tiles than
+// CTAs some shares are empty and wrote nothing, and those slots are skipped.
 template <bool FP16>
-__global__ void __launch_bounds__(128) attn_decode_combine_kernel(const float* __restrict__ part_o,
-                                                                  const float* __restrict__ part_lse, int nsplit,
-                                                                  int rows, void* o, float* lse) {
+__global__ void __launch_bounds__(128) attn_decode_combine_kernel(const DecParams p, int ctas, void* o, float* lse) {
   const int row = blockIdx.x, c = threadIdx.x;
-  float mx = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, __ldg(&part_lse[(size_t)s * rows + row]));
-  float wsum = 0.f, acc = 0.f;
-  if (mx != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float ls = __ldg(&part_lse[(size_t)s * rows + row]);
-      const float w = ls == -INFINITY ? 0.f : __expf(ls - mx);
+  const int per_b = p.Hq * p.Nq;
+  const int b = row / per_b, hq = (row - b * per_b) / p.Nq, i = row - b * per_b - hq * p.Nq;
+  const int G = p.Hq / p.Hkv;
+  const int u = b * p.Hkv + hq / G, col = (hq % G) * p.Nq + i;
+  float mx = -INFINITY, wsum = 0.f, acc = 0.f;
+  if (dec_len(p, b) > 0) {
+    const long long T = *p.total, P = ctas;
+    const int i0 = __ldg(&p.unit_first[u]);
+    const int n = __ldg(&p.unit_count[u]);
+    for (int s = 0; s < n; ++s) {
+      if (T < P && T * (i0 + s) / P == T * (i0 + s + 1) / P) continue;  // an empty share
+      const long long slot = (long long)u + i0 + s;
+      const float ls = __ldg(&p.part_lse[slot * p.R + col]);
+      const float ov = __ldg(&p.part_o[(slot * p.R + col) * 128 + c]);
+      if (ls == -INFINITY) continue;
+      if (ls > mx) {
+        const float sc = __expf(mx - ls);  // 0 for the first piece
+        acc *= sc;
+        wsum *= sc;
+        mx = ls;
+      }
+      const float w = __expf(ls - mx);
+      acc = fmaf(w, ov, acc);
       wsum += w;
-      acc = fmaf(w, __ldg(&part_o[((size_t)s * rows + row) * 128 + c]), acc);
     }
   }
-  const float val = wsum > 0.f ? acc / wsum : 0.f;
-  reinterpret_cast<uint16_t*>(o)[(size_t)row * 128 + c] = to16<FP16>(val);
+  reinterpret_cast<uint16_t*>(o)[(size_t)row * 128 + c] = to16<FP16>(wsum > 0.f ? acc / wsum : 0.f);
   if (lse != nullptr && c == 0) lse[row] = wsum > 0.f ? mx + __logf(wsum) : -INFINITY;
 }
 

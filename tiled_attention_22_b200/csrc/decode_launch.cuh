@@ -1,7 +1,7 @@
 #pragma once
-// decode_launch.cuh - host side of the KV-cache decode path: split count, workspace layout, TMA
-// descriptors and the two launches (split kernel, then the log-sum-exp merge when there is more
-// than one split).  Included by api.cu inside its anonymous namespace (after tma_host.cuh).
+// decode_launch.cuh - host side of the KV-cache decode path: CTA count, workspace layout, TMA
+// descriptors and the two launches (the persistent kernel, then the log-sum-exp merge of the
+// pieces).  Included by api.cu inside its anonymous namespace (after tma_host.cuh).
 
 // Query rows per kv head that the decode kernel takes: (Hq/Hkv) * Nq <= 64.
 constexpr int kDecodeMaxRows = 64;
@@ -25,34 +25,36 @@ int device_sm_count() {
   return n;
 }
 
-// Splits of each sequence's key range.  Requested > 0: that many (at most one per key tile).
-// 0: enough CTAs to give every SM one (batch, kv head, split), keeping at least 4 key tiles of
-// 128 per split so that each CTA's TMA ring reaches steady state.
-int decode_splits(int B, int Hkv, int Nk, int requested) {
-  const int tiles = (Nk + 127) / 128;
-  if (requested > 0) return std::min(requested, tiles);
-  const long long units = (long long)B * Hkv;
-  long long s = device_sm_count() / units;
-  s = std::min<long long>(s, std::max(1, tiles / 4));
-  return (int)std::max<long long>(1, s);
+// Persistent CTAs: requested > 0 takes that many, 0 one per SM; never more than there are key
+// tiles in the largest possible problem (B * Hkv units of ceil(Nk / 128) tiles).
+int decode_ctas(int B, int Hkv, int Nk, int requested) {
+  const long long tiles = (long long)B * Hkv * ((Nk + 127) / 128);
+  const long long want = requested > 0 ? requested : device_sm_count();
+  return (int)std::max<long long>(1, std::min(want, tiles));
 }
 
+// Workspace: the pieces' partial outputs and lse (slot = unit + CTA index, U + P - 1 slots), per
+// unit the first and the number of CTAs that may hold its pieces, and the total tile count.
 struct DecWs {
-  size_t part_o, part_lse, total;
+  size_t part_o, part_lse, unit_first, unit_count, tiles, total;
 };
 
-DecWs decode_ws(int B, int Hq, int Nq, int nsplit) {
+DecWs decode_ws(int B, int Hkv, int R, int P) {
+  const size_t U = (size_t)B * Hkv, slots = U + (size_t)P - 1;
   DecWs w{};
-  if (nsplit <= 1) return w;
-  const size_t rows = (size_t)B * Hq * Nq;
-  w.part_o = 0;
-  w.part_lse = align256((size_t)nsplit * rows * 128 * sizeof(float));
-  w.total = w.part_lse + align256((size_t)nsplit * rows * sizeof(float));
+  size_t off = 0;
+  w.part_o = off;     off += align256(slots * R * 128 * sizeof(float));
+  w.part_lse = off;   off += align256(slots * R * sizeof(float));
+  w.unit_first = off; off += align256(U * sizeof(int));
+  w.unit_count = off; off += align256(U * sizeof(int));
+  w.tiles = off;      off += 256;
+  w.total = off;
   return w;
 }
 
 template <int RP, bool FP16>
-int launch_decode_t(const void* q, const void* k, const void* v, const DecParams& p, cudaStream_t stream) {
+int launch_decode_t(const void* q, const void* k, const void* v, void* o, float* lse, int ctas, const DecParams& p,
+                    cudaStream_t stream) {
   using C = DecCfg<RP>;
   const CUtensorMapDataType dt = FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap tq, tk, tv;
@@ -71,35 +73,38 @@ int launch_decode_t(const void* q, const void* k, const void* v, const DecParams
     TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
     configured[dev].store(1, std::memory_order_release);
   }
-  const long long grid = (long long)p.B * p.Hkv * p.nsplit;
-  kern<<<(unsigned)grid, C::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  kern<<<(unsigned)ctas, C::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   TATTN_CUDA(cudaGetLastError());
-  if (p.nsplit > 1) {
-    const int rows = p.B * p.Hq * p.Nq;
-    attn_decode_combine_kernel<FP16><<<(unsigned)rows, 128, 0, stream>>>(p.part_o, p.part_lse, p.nsplit, rows, p.o,
-                                                                         p.lse);
-    TATTN_CUDA(cudaGetLastError());
-  }
+  const int rows = p.B * p.Hq * p.Nq;
+  attn_decode_combine_kernel<FP16><<<(unsigned)rows, 128, 0, stream>>>(p, ctas, o, lse);
+  TATTN_CUDA(cudaGetLastError());
   return ATTN_OK;
 }
 
-int launch_decode(const void* q, const void* k, const void* v, int dtype, const DecParams& p, cudaStream_t stream) {
+int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int dtype, int ctas,
+                  const DecParams& p, cudaStream_t stream) {
   const bool fp16 = dtype == ATTN_FP16;
   switch (decode_rp(p.R)) {
-    case 16: return fp16 ? launch_decode_t<16, true>(q, k, v, p, stream) : launch_decode_t<16, false>(q, k, v, p, stream);
-    case 32: return fp16 ? launch_decode_t<32, true>(q, k, v, p, stream) : launch_decode_t<32, false>(q, k, v, p, stream);
-    case 64: return fp16 ? launch_decode_t<64, true>(q, k, v, p, stream) : launch_decode_t<64, false>(q, k, v, p, stream);
+    case 16:
+      return fp16 ? launch_decode_t<16, true>(q, k, v, o, lse, ctas, p, stream)
+                  : launch_decode_t<16, false>(q, k, v, o, lse, ctas, p, stream);
+    case 32:
+      return fp16 ? launch_decode_t<32, true>(q, k, v, o, lse, ctas, p, stream)
+                  : launch_decode_t<32, false>(q, k, v, o, lse, ctas, p, stream);
+    case 64:
+      return fp16 ? launch_decode_t<64, true>(q, k, v, o, lse, ctas, p, stream)
+                  : launch_decode_t<64, false>(q, k, v, o, lse, ctas, p, stream);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
 
 // Argument checks shared by attn_decode and attn_decode_workspace_bytes.
-int check_decode_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || num_splits < 0) return ATTN_ERR_ARG;
+int check_decode_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1 || num_ctas < 0) return ATTN_ERR_ARG;
   if (Hq % Hkv || Nq > Nk) return ATTN_ERR_ARG;
   if (d != 128) return ATTN_ERR_UNSUPPORTED;
   if ((long long)(Hq / Hkv) * Nq > kDecodeMaxRows) return ATTN_ERR_UNSUPPORTED;
-  if ((long long)B * Hkv > (1 << 24) || Nk > (1 << 30) || (long long)B * Hq * Nq > (1 << 30) || num_splits > 4096)
+  if ((long long)B * Hkv > (1 << 24) || Nk > (1 << 30) || (long long)B * Hq * Nq > (1 << 30) || num_ctas > 65536)
     return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
