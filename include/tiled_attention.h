@@ -198,10 +198,13 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
  *   num_ctas: persistent CTAs (0: one per SM of the current device).  All key tiles of all
  *           (batch, kv head) units form one sequence, and CTA i of P takes the contiguous share
  *           [floor(i T / P), floor((i + 1) T / P)) of its T tiles, so ragged lengths stay
- *           balanced.  The part of a unit inside one CTA's share is a piece; a second, small
- *           kernel merges each unit's pieces by their log-sum-exp.
+ *           balanced.  The part of a unit inside one CTA's share is a piece; the CTA that
+ *           finishes a unit's last piece merges the pieces by their log-sum-exp (one launch).
  *   workspace: at least attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_ctas) bytes,
- *           16-byte aligned; its contents need no initialisation.
+ *           16-byte aligned, and ZEROED before its first use (e.g. cudaMemsetAsync): it holds
+ *           one arrival counter per (batch, kv head) at its start, which every completed call
+ *           leaves at zero again, so one zeroed workspace of the largest size needed serves
+ *           calls with any num_ctas.  After a call that ends in ATTN_ERR_TIMEOUT, zero it again.
  *   kv_lens must be 4-byte aligned; every other pointer 16-byte aligned.
  */
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas);

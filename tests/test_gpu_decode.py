@@ -185,3 +185,20 @@ def test_decode_workloads_full_size(ta, cfg):
     O, L, seen = expected(q, k, v, lt.tolist(), w.causal, w.scale, heads=heads)
     o, l = run(ta, q, k, v, lt, w.causal, 0, nan_tail=(w.lens != "full"))
     check(o, l, O, L, seen, w.name, heads=heads)
+
+
+def test_workspace_reuse_across_calls(ta):
+    """One zeroed workspace reused for several calls with different lengths and CTA counts: the
+    per-unit arrival counters must come back to zero after every call."""
+    q, k, v, _ = _inputs(3, 16, 4, 2, 3000, "bf16", "normal", 94000, None)
+    ws = torch.zeros(ta.attn_decode_workspace_bytes(3, 16, 4, 2, 3000, 128, 148), dtype=torch.uint8, device="cuda")
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    for lens, ctas in (([3000, 2000, 1000], 148), ([17, 2999, 640], 37), ([3000, 3000, 3000], 148), ([5, 0, 2500], 9)):
+        lt = torch.tensor(lens, dtype=torch.int32)
+        o, l = ta.attn_decode(qc, kc, vc, lt.cuda(), causal=True, num_ctas=ctas, workspace=ws)
+        torch.cuda.synchronize()
+        assert ta.attn_check_status() == 0
+        O, L, seen = expected(q, k, v, lens, True, 128 ** -0.5)
+        check(_np(o), l.cpu().numpy().astype(np.float64), O, L, seen, f"lens {lens} ctas {ctas}")
+    # the per-unit arrival counters (the first U int32 of the workspace) are back at zero
+    assert not ws[:3 * 4 * 4].cpu().numpy().any()

@@ -170,8 +170,8 @@ def attn_decode(q, k_cache, v_cache, kv_lens=None, causal=False, scale=None, num
     o = torch.empty_like(q) if out is None else out
     l = _lse_arg(lse, (B, Hq, Nq), q.device)
     ws_bytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_ctas)
-    if ws_bytes and workspace is None:
-        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    if ws_bytes and workspace is None:  # (a reused workspace must have been zeroed once)
+        workspace = torch.zeros(ws_bytes, device=q.device, dtype=torch.uint8)
     rc = lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kv_lens), _ptr(o), _ptr(l), B, Hq, Hkv, Nq,
                          Nk, d, int(bool(causal)), scale, DTYPES[q.dtype], int(num_ctas), _ptr(workspace),
                          0 if workspace is None else workspace.numel() * workspace.element_size(),

@@ -443,13 +443,13 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.kv_lens = kv_lens;
+  p.o = o;
+  p.lse = lse;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.part_o = reinterpret_cast<float*>(ws + w.part_o);
   p.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
-  p.unit_first = reinterpret_cast<int*>(ws + w.unit_first);
-  p.unit_count = reinterpret_cast<int*>(ws + w.unit_count);
-  p.total = reinterpret_cast<long long*>(ws + w.tiles);
-  return launch_decode(q, k_cache, v_cache, o, lse, dtype, ctas, p, static_cast<cudaStream_t>(stream));
+  p.unit_arrived = reinterpret_cast<unsigned int*>(ws + w.unit_arrived);
+  return launch_decode(q, k_cache, v_cache, dtype, ctas, p, static_cast<cudaStream_t>(stream));
 }
 
 int attn_check_status(void) {

@@ -49,13 +49,15 @@ struct DecParams {
   int causal;
   float scale_log2;      // scale * log2(e)
   const int* kv_lens;    // [B] cached keys per sequence (clamped to [0, Nk]); null: all Nk
-  // Partial results of the pieces (see the scheduling note in attn_decode_kernel): the piece of
-  // unit u processed by CTA i goes to slot u + i, so U + P - 1 slots cover every partition.
+  void* o;               // [B, Hq, Nq, 128] 16-bit
+  float* lse;            // [B, Hq, Nq] or null
+  // A unit split over several CTAs: each piece's partial result goes to slot u + i (CTA i), so
+  // U + P - 1 slots cover every partition, and the CTA that finishes the unit's last piece
+  // merges them (it learns that it is last from the unit's arrival counter, which it then resets
+  // to zero, so a completed call leaves every counter at zero).
   float* part_o;         // [slots, R, 128] fp32, normalised per piece
   float* part_lse;       // [slots, R]
-  int* unit_first;       // [U] the CTA holding each unit's first tile
-  int* unit_count;       // [U] CTAs from there to the one holding its last tile (some may be empty)
-  long long* total;      // [1] key tiles in all (written by CTA 0)
+  unsigned int* unit_arrived;  // [U]
 };
 
 template <int RP>
@@ -83,8 +85,8 @@ struct DecCfg {
   static constexpr int OFF_K = OFF_P + 2 * P_TILE;
   static constexpr int OFF_V = OFF_K + KS * KV_TILE;
   static constexpr int OFF_RED = OFF_V + VS * KV_TILE;    // float [2][4][RP]: per-warp column maxima
-  static constexpr int OFF_LRED = OFF_RED + 2 * RP * 16;  // float [RP][4]: per-warp row sums
-  static constexpr int OFF_M = OFF_LRED + RP * 16;        // float [2][RP]: running column maxima
+  static constexpr int OFF_LRED = OFF_RED + 2 * RP * 16;  // float [RP][4] per-warp row sums, + 1 flag
+  static constexpr int OFF_M = OFF_LRED + RP * 16 + 16;   // float [2][RP]: running column maxima
   static constexpr int OFF_SCHED = OFF_M + 2 * RP * 4;    // long long [8]: this CTA's tile range
   static constexpr int OFF_BAR = OFF_SCHED + 64;
   // q_full[2], q_empty[2], k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], s_free[2],
@@ -97,6 +99,7 @@ struct DecCfg {
   __host__ __device__ static constexpr uint32_t tm_o(int buf) { return (uint32_t)((2 + buf) * RP); }
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(RP % 16 == 0 && RP <= 64, "N of the M = 128 MMAs");
+  static_assert(CW % 8 == 0, "the merge takes columns eight at a time");
 };
 
 enum : int { WD_LOAD = 0x60, WD_MMA = 0x70, WD_SOFTMAX = 0x80, WD_DRAIN = 0x90 };
@@ -337,7 +340,6 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const long long total_tiles = sched[2];
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.total = total_tiles;
 
   if (warp == C::kTmaWarp) {
     // ================================ TMA producer ================================
@@ -453,7 +455,18 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
     const int t = wq * 32 + lane;    // TMEM lane: key t of the S^T tile, channel t of O^T
     const int c0 = wg * CW;          // first query column of this warpgroup
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const int bar_id = 1 + wg;
+    // one named barrier for all softmax warps: every decision taken on it is uniform across them
+    constexpr int kBar = 1, kBarThreads = C::kSoftmaxWarps * 32;
+    const int st = threadIdx.x;  // 0 .. kBarThreads - 1
+    // rows of sequences without keys: O = 0, lse = -inf (no piece covers them)
+    for (int bz = blockIdx.x; bz < p.B; bz += gridDim.x) {
+      if (dec_len(p, bz) > 0) continue;
+      const long long r0 = (long long)bz * p.Hq * p.Nq, nrow = (long long)p.Hq * p.Nq;
+      for (long long e = st; e < nrow * 128; e += kBarThreads)
+        reinterpret_cast<uint16_t*>(p.o)[r0 * 128 + e] = 0;
+      if (p.lse != nullptr)
+        for (long long e = st; e < nrow; e += kBarThreads) p.lse[r0 + e] = -INFINITY;
+    }
     // P^T store address of element (row c, key t): two 64-key panels, 128-byte swizzle
     const uint32_t p_base = smem_u32(sP) + (uint32_t)(t >> 6) * C::P_PANEL + (uint32_t)(t & 7) * 2;
     const uint32_t p_chunk = (uint32_t)((t & 63) >> 3);
@@ -512,7 +525,7 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
             dst[q4] = make_float4(wm[4 * q4], wm[4 * q4 + 1], wm[4 * q4 + 2], wm[4 * q4 + 3]);
         }
       }
-      if (!(ok = named_bar_and(bar_id, 128, okw && ok))) break;
+      if (!(ok = named_bar_and(kBar, kBarThreads, okw && ok))) break;
       // Column maxima over the 128 keys and the lazy update of the running max m (kept in shared
       // memory, double-buffered by tile parity: every thread computes the same m, one thread
       // stores it).  Then P^T = exp2(s * scale_log2 - m), with masked keys giving exp2(-inf) = 0,
@@ -609,32 +622,114 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
           for (int sh = 16; sh > 0; sh >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sh);
           if (lane == 0) lred[(c0 + r) * 4 + wq] = v;
         }
-        if (!(ok = named_bar_and(bar_id, 128, oke))) break;
+        if (!(ok = named_bar_and(kBar, kBarThreads, oke))) break;
         tc_fence_after();
         uint32_t o[CW];
         tmem_ld_cols<CW>(tmem + C::tm_o(ob) + (uint32_t)c0 + lane_off, o);
         const int u = cur.unit(p);
-        const long long slot = (long long)u + blockIdx.x;
         const float* m_last = m_sh + buf * RP;
+        const long long row0 = (long long)u * p.R;  // output row of column 0 ((b, h, i) order)
+        if (cur.ps == 0 && cur.pe == cur.ntb) {
+          // the whole unit is this piece: final output
 #pragma unroll
-        for (int r = 0; r < CW; ++r) {
-          const int c = c0 + r;
-          if (c < p.R) {
-            const float4 l4 = *reinterpret_cast<const float4*>(&lred[c * 4]);
-            const float lsum = (l4.x + l4.y) + (l4.z + l4.w);
-            p.part_o[(slot * p.R + c) * 128 + t] = lsum > 0.f ? __uint_as_float(o[r]) / lsum : 0.f;
-            if (t == r)
-              p.part_lse[slot * p.R + c] =
-                  lsum > 0.f ? (m_last[c] + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+          for (int r = 0; r < CW; ++r) {
+            const int c = c0 + r;
+            if (c < p.R) {
+              const float4 l4 = *reinterpret_cast<const float4*>(&lred[c * 4]);
+              const float lsum = (l4.x + l4.y) + (l4.z + l4.w);
+              reinterpret_cast<uint16_t*>(p.o)[(row0 + c) * 128 + t] =
+                  to16<FP16>(lsum > 0.f ? __uint_as_float(o[r]) / lsum : 0.f);
+              if (p.lse != nullptr && t == r)
+                p.lse[row0 + c] = lsum > 0.f ? (m_last[c] + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+            }
           }
-        }
-        if (cur.ps == 0 && threadIdx.x == 0) {
-          // this CTA holds the unit's first tile: record which CTAs hold its pieces.  The unit's
-          // last tile lies in CTA ceil((g_u + n) P / T) - 1, g_u being its first global tile.
-          const long long gu = cur.g - cur.lt, P = gridDim.x;
-          const long long i_last = ((gu + cur.ntb) * P + total_tiles - 1) / total_tiles - 1;
-          p.unit_first[u] = (int)blockIdx.x;
-          p.unit_count[u] = (int)(i_last - blockIdx.x + 1);
+        } else {
+          // a part of the unit: partial output (normalised) and lse to slot u + CTA index
+          const long long slot = (long long)u + blockIdx.x;
+#pragma unroll
+          for (int r = 0; r < CW; ++r) {
+            const int c = c0 + r;
+            if (c < p.R) {
+              const float4 l4 = *reinterpret_cast<const float4*>(&lred[c * 4]);
+              const float lsum = (l4.x + l4.y) + (l4.z + l4.w);
+              p.part_o[(slot * p.R + c) * 128 + t] = lsum > 0.f ? __uint_as_float(o[r]) / lsum : 0.f;
+              if (t == r)
+                p.part_lse[slot * p.R + c] =
+                    lsum > 0.f ? (m_last[c] + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+            }
+          }
+          __threadfence();  // this thread's partials are visible GPU-wide before the arrival below
+          // The unit's tiles [g_u, g_u + n) lie in the CTAs i(g_u) .. i(g_u + n - 1), with
+          // i(x) = ceil((x + 1) P / T) - 1; with fewer tiles than CTAs, empty shares hold nothing.
+          const long long T = total_tiles, P = gridDim.x, gu = cur.g - cur.lt;
+          const long long i_first = ((gu + 1) * P + T - 1) / T - 1;
+          const long long i_last = ((gu + cur.ntb) * P + T - 1) / T - 1;
+          named_bar_sync(kBar, kBarThreads);
+          if (st == 0) {
+            long long pieces = i_last - i_first + 1;
+            if (T < P)
+              for (long long i = i_first; i <= i_last; ++i) pieces -= (T * i / P == T * (i + 1) / P) ? 1 : 0;
+            const unsigned int arrived = atomicAdd(&p.unit_arrived[u], 1u) + 1u;
+            const bool last = arrived == (unsigned int)pieces;
+            if (last) {
+              p.unit_arrived[u] = 0u;  // every piece has arrived: nothing else touches it this call
+              __threadfence();
+            }
+            lred[4 * RP] = last ? 1.f : 0.f;
+          }
+          named_bar_sync(kBar, kBarThreads);
+          if (lred[4 * RP] != 0.f) {
+            // merge: O = sum_i w_i O_i / sum_i w_i, w_i = exp(lse_i - max), lse = max + log(sum_i w_i),
+            // running max over the pieces; 8 columns x 4 pieces of loads in flight at a time
+            constexpr int MG = 8, KP = 4;
+            for (int cg = 0; cg < CW; cg += MG) {
+              float mx[MG], wsum[MG], acc[MG];
+#pragma unroll
+              for (int r = 0; r < MG; ++r) { mx[r] = -INFINITY; wsum[r] = 0.f; acc[r] = 0.f; }
+              for (long long i = i_first; i <= i_last; i += KP) {
+                float ls[KP][MG], ov[KP][MG];
+#pragma unroll
+                for (int kp = 0; kp < KP; ++kp) {
+                  const long long ii = i + kp;
+                  const bool have = ii <= i_last && !(T < P && T * ii / P == T * (ii + 1) / P);
+                  const long long sl = (long long)u + ii;
+#pragma unroll
+                  for (int r = 0; r < MG; ++r) {
+                    const int c = c0 + cg + r;
+                    const bool use = have && c < p.R;
+                    ls[kp][r] = use ? __ldcg(&p.part_lse[sl * p.R + c]) : -INFINITY;
+                    ov[kp][r] = use ? __ldcg(&p.part_o[(sl * p.R + c) * 128 + t]) : 0.f;
+                  }
+                }
+#pragma unroll
+                for (int kp = 0; kp < KP; ++kp)
+#pragma unroll
+                  for (int r = 0; r < MG; ++r) {
+                    const float l_i = ls[kp][r];
+                    if (l_i == -INFINITY) continue;
+                    if (l_i > mx[r]) {
+                      const float sc = __expf(mx[r] - l_i);  // 0 for the first piece
+                      acc[r] *= sc;
+                      wsum[r] *= sc;
+                      mx[r] = l_i;
+                    }
+                    const float w = __expf(l_i - mx[r]);
+                    acc[r] = fmaf(w, ov[kp][r], acc[r]);
+                    wsum[r] += w;
+                  }
+              }
+#pragma unroll
+              for (int r = 0; r < MG; ++r) {
+                const int c = c0 + cg + r;
+                if (c < p.R) {
+                  reinterpret_cast<uint16_t*>(p.o)[(row0 + c) * 128 + t] =
+                      to16<FP16>(wsum[r] > 0.f ? acc[r] / wsum[r] : 0.f);
+                  if (p.lse != nullptr && t == 0)
+                    p.lse[row0 + c] = wsum[r] > 0.f ? mx[r] + __logf(wsum[r]) : -INFINITY;
+                }
+              }
+            }
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -651,44 +746,6 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-}
-
-// Merge of the pieces of one query row: O = sum_s w_s O_s / sum_s w_s with w_s = exp(lse_s - max),
-// lse = max + log(sum_s w_s), in one pass with a running max.  One CTA of 128 threads (one per
-// channel) per row; a row whose sequence holds no key gets O = 0 and lse = -inf.  The pieces of
-// unit u are in slots u + i for the CTAs i from unit_first[u] on; when there are fewer tiles than
-// CTAs some shares are empty and wrote nothing, and those slots are skipped.
-template <bool FP16>
-__global__ void __launch_bounds__(128) attn_decode_combine_kernel(const DecParams p, int ctas, void* o, float* lse) {
-  const int row = blockIdx.x, c = threadIdx.x;
-  const int per_b = p.Hq * p.Nq;
-  const int b = row / per_b, hq = (row - b * per_b) / p.Nq, i = row - b * per_b - hq * p.Nq;
-  const int G = p.Hq / p.Hkv;
-  const int u = b * p.Hkv + hq / G, col = (hq % G) * p.Nq + i;
-  float mx = -INFINITY, wsum = 0.f, acc = 0.f;
-  if (dec_len(p, b) > 0) {
-    const long long T = *p.total, P = ctas;
-    const int i0 = __ldg(&p.unit_first[u]);
-    const int n = __ldg(&p.unit_count[u]);
-    for (int s = 0; s < n; ++s) {
-      if (T < P && T * (i0 + s) / P == T * (i0 + s + 1) / P) continue;  // an empty share
-      const long long slot = (long long)u + i0 + s;
-      const float ls = __ldg(&p.part_lse[slot * p.R + col]);
-      const float ov = __ldg(&p.part_o[(slot * p.R + col) * 128 + c]);
-      if (ls == -INFINITY) continue;
-      if (ls > mx) {
-        const float sc = __expf(mx - ls);  // 0 for the first piece
-        acc *= sc;
-        wsum *= sc;
-        mx = ls;
-      }
-      const float w = __expf(ls - mx);
-      acc = fmaf(w, ov, acc);
-      wsum += w;
-    }
-  }
-  reinterpret_cast<uint16_t*>(o)[(size_t)row * 128 + c] = to16<FP16>(wsum > 0.f ? acc / wsum : 0.f);
-  if (lse != nullptr && c == 0) lse[row] = wsum > 0.f ? mx + __logf(wsum) : -INFINITY;
 }
 
 }  // namespace tattn

@@ -1,7 +1,6 @@
 #pragma once
 // decode_launch.cuh - host side of the KV-cache decode path: CTA count, workspace layout, TMA
-// descriptors and the two launches (the persistent kernel, then the log-sum-exp merge of the
-// pieces).  Included by api.cu inside its anonymous namespace (after tma_host.cuh).
+// descriptors and the launch of the persistent kernel (which also merges the pieces).  Included by api.cu inside its anonymous namespace (after tma_host.cuh).
 
 // Query rows per kv head that the decode kernel takes: (Hq/Hkv) * Nq <= 64.
 constexpr int kDecodeMaxRows = 64;
@@ -33,28 +32,27 @@ int decode_ctas(int B, int Hkv, int Nk, int requested) {
   return (int)std::max<long long>(1, std::min(want, tiles));
 }
 
-// Workspace: the pieces' partial outputs and lse (slot = unit + CTA index, U + P - 1 slots), per
-// unit the first and the number of CTAs that may hold its pieces, and the total tile count.
+// Workspace: one arrival counter per unit (zero between calls), then the pieces' partial outputs
+// and lse (slot = unit + CTA index, U + P - 1 slots).
 struct DecWs {
-  size_t part_o, part_lse, unit_first, unit_count, tiles, total;
+  size_t part_o, part_lse, unit_arrived, total;
 };
 
 DecWs decode_ws(int B, int Hkv, int R, int P) {
   const size_t U = (size_t)B * Hkv, slots = U + (size_t)P - 1;
   DecWs w{};
   size_t off = 0;
-  w.part_o = off;     off += align256(slots * R * 128 * sizeof(float));
-  w.part_lse = off;   off += align256(slots * R * sizeof(float));
-  w.unit_first = off; off += align256(U * sizeof(int));
-  w.unit_count = off; off += align256(U * sizeof(int));
-  w.tiles = off;      off += 256;
+  // the counters come first, so that their place does not depend on the CTA count and one
+  // zeroed workspace serves calls with any count that fits
+  w.unit_arrived = off; off += align256(U * sizeof(unsigned int));
+  w.part_o = off;       off += align256(slots * R * 128 * sizeof(float));
+  w.part_lse = off;     off += align256(slots * R * sizeof(float));
   w.total = off;
   return w;
 }
 
 template <int RP, bool FP16>
-int launch_decode_t(const void* q, const void* k, const void* v, void* o, float* lse, int ctas, const DecParams& p,
-                    cudaStream_t stream) {
+int launch_decode_t(const void* q, const void* k, const void* v, int ctas, const DecParams& p, cudaStream_t stream) {
   using C = DecCfg<RP>;
   const CUtensorMapDataType dt = FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap tq, tk, tv;
@@ -75,25 +73,19 @@ int launch_decode_t(const void* q, const void* k, const void* v, void* o, float*
   }
   kern<<<(unsigned)ctas, C::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   TATTN_CUDA(cudaGetLastError());
-  const int rows = p.B * p.Hq * p.Nq;
-  attn_decode_combine_kernel<FP16><<<(unsigned)rows, 128, 0, stream>>>(p, ctas, o, lse);
-  TATTN_CUDA(cudaGetLastError());
   return ATTN_OK;
 }
 
-int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int dtype, int ctas,
-                  const DecParams& p, cudaStream_t stream) {
+int launch_decode(const void* q, const void* k, const void* v, int dtype, int ctas, const DecParams& p,
+                  cudaStream_t stream) {
   const bool fp16 = dtype == ATTN_FP16;
   switch (decode_rp(p.R)) {
     case 16:
-      return fp16 ? launch_decode_t<16, true>(q, k, v, o, lse, ctas, p, stream)
-                  : launch_decode_t<16, false>(q, k, v, o, lse, ctas, p, stream);
+      return fp16 ? launch_decode_t<16, true>(q, k, v, ctas, p, stream) : launch_decode_t<16, false>(q, k, v, ctas, p, stream);
     case 32:
-      return fp16 ? launch_decode_t<32, true>(q, k, v, o, lse, ctas, p, stream)
-                  : launch_decode_t<32, false>(q, k, v, o, lse, ctas, p, stream);
+      return fp16 ? launch_decode_t<32, true>(q, k, v, ctas, p, stream) : launch_decode_t<32, false>(q, k, v, ctas, p, stream);
     case 64:
-      return fp16 ? launch_decode_t<64, true>(q, k, v, o, lse, ctas, p, stream)
-                  : launch_decode_t<64, false>(q, k, v, o, lse, ctas, p, stream);
+      return fp16 ? launch_decode_t<64, true>(q, k, v, ctas, p, stream) : launch_decode_t<64, false>(q, k, v, ctas, p, stream);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
