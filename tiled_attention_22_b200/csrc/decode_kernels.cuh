@@ -658,23 +658,22 @@ __global__ void __launch_bounds__(DecCfg<RP>::kThreads, 1)
                     lsum > 0.f ? (m_last[c] + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
             }
           }
-          __threadfence();  // this thread's partials are visible GPU-wide before the arrival below
           // The unit's tiles [g_u, g_u + n) lie in the CTAs i(g_u) .. i(g_u + n - 1), with
           // i(x) = ceil((x + 1) P / T) - 1; with fewer tiles than CTAs, empty shares hold nothing.
           const long long T = total_tiles, P = gridDim.x, gu = cur.g - cur.lt;
           const long long i_first = ((gu + 1) * P + T - 1) / T - 1;
           const long long i_last = ((gu + cur.ntb) * P + T - 1) / T - 1;
+          // The barrier orders every thread's partial stores before thread 0's arrival, whose
+          // release (cumulative over what the barrier ordered) publishes them GPU-wide; its
+          // acquire makes the other pieces' partials visible to the CTA's merge below.
           named_bar_sync(kBar, kBarThreads);
           if (st == 0) {
             long long pieces = i_last - i_first + 1;
             if (T < P)
               for (long long i = i_first; i <= i_last; ++i) pieces -= (T * i / P == T * (i + 1) / P) ? 1 : 0;
-            const unsigned int arrived = atomicAdd(&p.unit_arrived[u], 1u) + 1u;
+            const unsigned int arrived = atom_add_acq_rel_gpu(&p.unit_arrived[u], 1u) + 1u;
             const bool last = arrived == (unsigned int)pieces;
-            if (last) {
-              p.unit_arrived[u] = 0u;  // every piece has arrived: nothing else touches it this call
-              __threadfence();
-            }
+            if (last) p.unit_arrived[u] = 0u;  // every piece has arrived: nothing else touches it this call
             lred[4 * RP] = last ? 1.f : 0.f;
           }
           named_bar_sync(kBar, kBarThreads);
