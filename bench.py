@@ -34,7 +34,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from attn_workloads import WORKLOADS, make_inputs  # noqa: E402
+from attn_workloads import DECODE_WORKLOADS, WORKLOADS, decode_bytes, make_decode_inputs, make_inputs  # noqa: E402
 
 
 KERNEL_SOURCES = ("tiled_attention_22_b200/csrc/attn_fwd_kernels.cuh", "tiled_attention_22_b200/csrc/ptx.cuh",
@@ -392,9 +392,55 @@ def run_native(args, w, world, rank, local):
     }
     if e2e:
         line["e2e"] = e2e
+    if not args.no_decode:
+        line["decode"] = run_decode(args, dev, world, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     return line
+
+
+def run_decode(args, dev, world, peaks):
+    """KV-cache decode (attn_decode) on the named decode workloads: device time of back-to-back
+    calls (every call reads its whole cache, 0.18-2.1 GB, larger than L2), bandwidth over the
+    algorithmic bytes (used K and V once, q and o), against the measured HBM copy bandwidth."""
+    import tiled_attention_22_b200 as ta
+
+    out = {}
+    for cfg, w in DECODE_WORKLOADS.items():
+        q, k, v, lens = make_decode_inputs(w)
+        q, k, v, lens_d = q.to(dev), k.to(dev), v.to(dev), lens.to(dev)
+        ws = torch.zeros(ta.attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, 0), device=dev,
+                         dtype=torch.uint8)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.Nq), device=dev, dtype=torch.float32)
+
+        def call():
+            ta.attn_decode(q, k, v, lens_d, causal=w.causal, scale=w.scale, out=o, lse=lse, workspace=ws)
+
+        for _ in range(max(3, args.warmup)):
+            call()
+        torch.cuda.synchronize()
+        _barrier(world)
+        n = 50
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        _barrier(world)
+        ms = _max_over_ranks(e0.elapsed_time(e1), world, dev) / n
+        if ta.attn_check_status() != 0:
+            raise RuntimeError("device-side wait timed out in the decode benchmark")
+        nbytes = decode_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.d, lens.tolist())
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[w.name] = {"ms_per_call": ms, "GB/s": gbs * world, "frac_of_hbm_peak": gbs / peaks["hbm_gbs"],
+                       "bytes_per_call": nbytes, "calls": n, "kernel": "attn_decode_kernel<16,bf16>",
+                       "launches_per_call": 1}
+        del q, k, v, o, ws
+        torch.cuda.empty_cache()
+    out["peak_note"] = "HBM copy bandwidth %.0f GB/s (%s)" % (peaks["hbm_gbs"], peaks["source"])
+    return out
 
 
 def _fused_bytes(w, mode):
@@ -425,6 +471,7 @@ def main():
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurements")
     ap.add_argument("--modes", default="int8_qk,bf16_exact",
                     help="modes to time (the headline value is int8_qk; drop one only for profiling)")
     args = ap.parse_args()
