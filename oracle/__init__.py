@@ -7,7 +7,9 @@ the CUDA path (no kernels, tables, helpers or constants); the only thing the
 two sides have in common is the seeded input generator in ``attn_workloads``.
 
 Contents
-  exact            O1: plain float64 softmax attention (the definition).
+  exact            O1: plain float64 softmax attention (the definition), also
+                   with Nq < Nk (queries after a KV cache) and with a per-row
+                   visible key prefix (the APB mask shape).
   int8_emulation   O2: bit-exact emulation of K smoothing and per-block INT8
                    quantisation of Q and K, exact integer QK^T, and the
                    float64 attention that follows from those quantised scores.
@@ -26,7 +28,7 @@ print no value for it.  The quantiser's constants and rounding are a reading of
 the pages (they are silent on them), so O2 is pinned to that reading, not to a
 number the pages print.
 """
-from .exact import attention, attention_probs, logsumexp_rows  # noqa: F401
+from .exact import attention, attention_prefix, attention_probs, logsumexp_rows  # noqa: F401
 from .int8_emulation import (  # noqa: F401
     QBLOCK,
     k_channel_mean,

@@ -95,3 +95,43 @@ def attention(q, k, v, scale, causal, rows=None):
             O[b, h] = (P @ v[b, g]) / l
             L[b, h] = m[:, 0] + np.log(l[:, 0])
     return O, L
+
+
+def attention_prefix(q, k, v, scale, row_limit, rows=None):
+    """O and lse with a per-query-row visible key prefix: query row i sees keys j < row_limit[i]
+    (the same limits for every batch and head), in float64.
+
+    This is the mask shape of the APB article ("在长文本上比Flash Attention快10倍！清华等提出APB序列
+    并行推理框架", sections on the anchor block, the passing block and the computation step: a
+    special FlashAttention kernel with a changed mask).  With the keys laid out as
+    [anchor | passing | local] and the queries as [anchor | local], an anchor query sees the
+    anchor causally and a local query sees the whole anchor and passing blocks and the local block
+    causally; both are prefixes of the key sequence (``apb_row_limits`` in the tests builds them).
+    Plain causal attention is row_limit[i] = i + 1.
+
+    Limits are clamped to [0, Nk].  A row with limit 0 sees no key; its softmax is empty and it is
+    reported as O = 0, lse = -inf (the same convention as the KV-cache decode path).
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; row_limit: [Nq] integers.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    lim = np.clip(np.asarray(row_limit, dtype=np.int64).reshape(-1), 0, Nk)
+    if lim.shape[0] != Nq:
+        raise ValueError("row_limit needs one entry per query row")
+    rows = np.arange(Nq) if rows is None else np.asarray(rows)
+    O = np.zeros((B, Hq, len(rows), v.shape[3]))
+    L = np.full((B, Hq, len(rows)), -np.inf)
+    visible = np.arange(Nk)[None, :] < lim[rows][:, None]
+    seen = visible.any(axis=1)
+    for b in range(B):
+        for h in range(Hq):
+            g = _kv_head(h, Hq, Hkv)
+            S = np.where(visible, scale * (q[b, h][rows] @ k[b, g].T), -np.inf)[seen]
+            m = S.max(axis=1, keepdims=True)
+            P = np.exp(S - m)
+            l = P.sum(axis=1, keepdims=True)
+            O[b, h, seen] = (P @ v[b, g]) / l
+            L[b, h, seen] = m[:, 0] + np.log(l[:, 0])
+    return O, L
+

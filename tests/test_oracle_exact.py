@@ -245,3 +245,95 @@ def test_short_queries_equal_the_last_rows_of_full_self_attention():
     O1c, _ = oracle.attention(q[:, :, -1:], k, v, 0.3, True)
     O1n, _ = oracle.attention(q[:, :, -1:], k, v, 0.3, False)
     np.testing.assert_array_equal(O1c, O1n)
+
+
+# ---------------------------------------------------------------------------------------------
+# Per-row visible key prefix (the APB mask shape)
+# ---------------------------------------------------------------------------------------------
+def apb_mask_blockwise(A, Pb, L):
+    """The APB mask written block by block from the article's description, independent of any
+    limit formula: keys [anchor A | passing Pb | local L], queries [anchor A | local L].  Anchor
+    queries see the anchor block causally; local queries see the anchor and passing blocks in
+    full and the local block causally."""
+    Nq, Nk = A + L, A + Pb + L
+    M = np.zeros((Nq, Nk), dtype=bool)
+    M[:A, :A] = np.tril(np.ones((A, A), dtype=bool))            # anchor x anchor: causal
+    M[A:, :A] = True                                            # local x anchor: full
+    M[A:, A:A + Pb] = True                                      # local x passing: full
+    M[A:, A + Pb:] = np.tril(np.ones((L, L), dtype=bool))       # local x local: causal
+    return M
+
+
+def apb_limits(A, Pb, L):
+    return np.concatenate([np.arange(1, A + 1), A + Pb + np.arange(1, L + 1)])
+
+
+@pytest.mark.parametrize("A,Pb,L", [(2, 3, 4), (1, 0, 5), (3, 5, 1), (4, 4, 4)])
+def test_apb_block_mask_is_a_row_prefix(A, Pb, L):
+    """Every row of the block-built APB mask is a prefix of the key sequence, of the length the
+    limit formula gives."""
+    M = apb_mask_blockwise(A, Pb, L)
+    lim = apb_limits(A, Pb, L)
+    assert np.array_equal(M, np.arange(A + Pb + L)[None, :] < lim[:, None])
+
+
+@pytest.mark.parametrize("A,Pb,L", [(2, 3, 4), (3, 0, 3)])
+def test_prefix_brute_force_apb(A, Pb, L):
+    q = RNG.standard_normal((1, 4, A + L, 5))
+    k = RNG.standard_normal((1, 2, A + Pb + L, 5))
+    v = RNG.standard_normal((1, 2, A + Pb + L, 3))
+    M = apb_mask_blockwise(A, Pb, L)
+    O, Lse = oracle.attention_prefix(q, k, v, 0.6, apb_limits(A, Pb, L))
+    for h in range(4):
+        g = h // 2
+        for i in range(A + L):
+            js = [j for j in range(A + Pb + L) if M[i, j]]
+            s = [0.6 * sum(float(q[0, h, i, c]) * float(k[0, g, j, c]) for c in range(5)) for j in js]
+            m = max(s)
+            w = [math.exp(x - m) for x in s]
+            tot = math.fsum(w)
+            for c in range(3):
+                ref = math.fsum(w[t] * float(v[0, g, j, c]) for t, j in enumerate(js)) / tot
+                assert abs(O[0, h, i, c] - ref) <= 1e-12
+            assert abs(Lse[0, h, i] - (m + math.log(tot))) <= 1e-12
+
+
+def test_prefix_matches_torch_sdpa_with_block_mask():
+    A, Pb, L = 48, 80, 200
+    g = torch.Generator().manual_seed(21)
+    q = torch.randn(2, 8, A + L, 64, generator=g, dtype=torch.float64)
+    k = torch.randn(2, 2, A + Pb + L, 64, generator=g, dtype=torch.float64)
+    v = torch.randn(2, 2, A + Pb + L, 64, generator=g, dtype=torch.float64)
+    M = torch.from_numpy(apb_mask_blockwise(A, Pb, L))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q, k.repeat_interleave(4, dim=1), v.repeat_interleave(4, dim=1), attn_mask=M, scale=0.125)
+    O, _ = oracle.attention_prefix(q, k, v, 0.125, apb_limits(A, Pb, L))
+    np.testing.assert_allclose(O, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_prefix_reduces_to_causal_and_full():
+    q = RNG.standard_normal((1, 2, 37, 8))
+    k = RNG.standard_normal((1, 2, 37, 8))
+    v = RNG.standard_normal((1, 2, 37, 8))
+    Oc, Lc = oracle.attention(q, k, v, 0.4, True)
+    Op, Lp = oracle.attention_prefix(q, k, v, 0.4, np.arange(1, 38))
+    np.testing.assert_array_equal(Op, Oc)
+    np.testing.assert_array_equal(Lp, Lc)
+    On, Ln = oracle.attention(q, k, v, 0.4, False)
+    Of, Lf = oracle.attention_prefix(q, k, v, 0.4, np.full(37, 10 ** 6))  # clamped to Nk
+    np.testing.assert_array_equal(Of, On)
+    np.testing.assert_array_equal(Lf, Ln)
+
+
+def test_prefix_empty_rows_and_row_subset():
+    q = RNG.standard_normal((1, 1, 6, 4))
+    k = RNG.standard_normal((1, 1, 9, 4))
+    v = RNG.standard_normal((1, 1, 9, 4))
+    lim = np.array([0, 3, 0, 9, 1, -5])
+    O, L = oracle.attention_prefix(q, k, v, 1.0, lim)
+    for i in (0, 2, 5):
+        assert (O[0, 0, i] == 0).all() and L[0, 0, i] == -np.inf
+    np.testing.assert_allclose(O[0, 0, 4], v[0, 0, 0], atol=1e-15)  # one visible key: its value
+    Os, Ls = oracle.attention_prefix(q, k, v, 1.0, lim, rows=[3, 1])
+    np.testing.assert_array_equal(Os[0, 0], O[0, 0, [3, 1]])
+    np.testing.assert_array_equal(Ls[0, 0], L[0, 0, [3, 1]])
