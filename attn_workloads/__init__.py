@@ -27,7 +27,8 @@ import math
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "attention_flops", "workload", "DecodeWorkload",
-           "DECODE_WORKLOADS", "make_decode_inputs", "decode_bytes"]
+           "DECODE_WORKLOADS", "make_decode_inputs", "decode_bytes", "ApbWorkload", "APB_WORKLOADS",
+           "make_apb_inputs"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -188,3 +189,59 @@ def decode_bytes(B: int, Hq: int, Hkv: int, Nq: int, d: int, lens) -> float:
     lengths x Hkv x d each), the queries and the outputs; every byte once."""
     total_len = float(sum(int(x) for x in lens))
     return 2.0 * 2.0 * total_len * Hkv * d + 2.0 * 2.0 * B * Hq * Nq * d
+
+
+# ------------------------------------------------------------------------------------------------
+# APB-shaped prefill on one device: keys [anchor A | passing P | local L], queries [anchor A |
+# local L] (the APB article's layout; the anchor block is 1/4 to 1/8 of the local block).
+# Recipe: q [B, Hq, A + L, d] and k, v [B, Hkv, A + P + L, d] drawn as above (seeds
+# seed_base + {0, 1, 2}, float32 N(0, 1), cast).
+# ------------------------------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class ApbWorkload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    anchor: int
+    passing: int
+    local: int
+    d: int
+    dtype: str
+    seed_base: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def torch_dtype(self):
+        return {"bf16": torch.bfloat16, "fp16": torch.float16}[self.dtype]
+
+    @property
+    def Nq(self) -> int:
+        return self.anchor + self.local
+
+    @property
+    def Nk(self) -> int:
+        return self.anchor + self.passing + self.local
+
+
+# 201: a 16K-token local block with an anchor of 1/8 of it and a 4K-token passing block (the
+#      compressed context of earlier devices), LLaMA-3-8B-shaped GQA heads.
+APB_WORKLOADS = {
+    201: ApbWorkload("apb_b1_hq32_hkv8_anchor2048_passing4096_local16384_d128", 1, 32, 8, 2048, 4096, 16384, 128,
+                     "bf16", 201000),
+}
+
+
+def make_apb_inputs(w: ApbWorkload):
+    """Return (q, k, v) as CPU tensors: q [B, Hq, anchor + local, d], k and v
+    [B, Hkv, anchor + passing + local, d]."""
+    f32 = torch.float32
+    q = torch.randn((w.B, w.Hq, w.Nq, w.d), generator=_gen(w.seed_base + 0), dtype=f32)
+    k = torch.randn((w.B, w.Hkv, w.Nk, w.d), generator=_gen(w.seed_base + 1), dtype=f32)
+    v = torch.randn((w.B, w.Hkv, w.Nk, w.d), generator=_gen(w.seed_base + 2), dtype=f32)
+    dt = w.torch_dtype
+    return q.to(dt), k.to(dt), v.to(dt)
+

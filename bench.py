@@ -34,7 +34,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from attn_workloads import DECODE_WORKLOADS, WORKLOADS, decode_bytes, make_decode_inputs, make_inputs  # noqa: E402
+from attn_workloads import (APB_WORKLOADS, DECODE_WORKLOADS, WORKLOADS, decode_bytes, make_apb_inputs,  # noqa: E402
+                            make_decode_inputs, make_inputs)
 
 
 KERNEL_SOURCES = ("tiled_attention_22_b200/csrc/attn_fwd_kernels.cuh", "tiled_attention_22_b200/csrc/ptx.cuh",
@@ -394,6 +395,7 @@ def run_native(args, w, world, rank, local):
         line["e2e"] = e2e
     if not args.no_decode:
         line["decode"] = run_decode(args, dev, world, peaks)
+        line["prefix_mask"] = run_prefix_mask(args, dev, world, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     return line
@@ -440,6 +442,48 @@ def run_decode(args, dev, world, peaks):
         del q, k, v, o, ws
         torch.cuda.empty_cache()
     out["peak_note"] = "HBM copy bandwidth %.0f GB/s (%s)" % (peaks["hbm_gbs"], peaks["source"])
+    return out
+
+
+def run_prefix_mask(args, dev, world, peaks):
+    """Row-prefix-masked forward (attn_fwd_prefix_masked) on the APB-shaped workload: device time
+    of back-to-back calls (inputs larger than L2), TFLOP/s over the visible (query, key) pairs
+    (4 d FLOPs each), against the measured bf16 GEMM rate."""
+    import tiled_attention_22_b200 as ta
+
+    out = {}
+    for cfg, w in APB_WORKLOADS.items():
+        q, k, v = (t.to(dev) for t in make_apb_inputs(w))
+        lim = ta.apb_row_limits(w.anchor, w.passing, w.local, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.Nq), device=dev, dtype=torch.float32)
+        flops = 4.0 * w.B * w.Hq * w.d * float(lim.clamp(0, w.Nk).sum().item())
+
+        def call():
+            ta.attn_fwd_prefix_masked(q, k, v, lim, scale=w.scale, out=o, lse=lse)
+
+        for _ in range(max(3, args.warmup)):
+            call()
+        torch.cuda.synchronize()
+        _barrier(world)
+        n = 20
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        _barrier(world)
+        ms = _max_over_ranks(e0.elapsed_time(e1), world, dev) / n
+        if ta.attn_check_status() != 0:
+            raise RuntimeError("device-side wait timed out in the prefix-mask benchmark")
+        tf = flops / (ms * 1e-3) / 1e12
+        out[w.name] = {"ms_per_call": ms, "TFLOP/s": tf * world, "frac_of_bf16_peak": tf / peaks["bf16"],
+                       "flops_per_call": flops, "calls": n, "kernel": "attn_fwd_kernel<128,bf16>",
+                       "launches_per_call": 1}
+        del q, k, v, o
+        torch.cuda.empty_cache()
+    out["peak_note"] = "bf16 dense GEMM %.0f TFLOP/s (%s, burst)" % (peaks["bf16"], peaks["source"])
     return out
 
 

@@ -179,6 +179,23 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
                   int dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * attn_fwd_prefix_masked - attention in which query row i sees the keys j < row_kv_limit[i]
+ * (a per-row visible prefix; the same limits for every batch and head), bf16/fp16 exact mode.
+ * This is the mask of the APB article ("在长文本上比Flash Attention快10倍！清华等提出APB序列并行推理
+ * 框架", sections on the anchor block, the passing block and the computation step, which uses a
+ * special FlashAttention kernel with a changed mask): with keys laid out as
+ * [anchor A | passing P | local L] and queries as [anchor A | local L], anchor row i has limit
+ * i + 1 and local row i has limit A + P + i + 1.  Plain causal attention is limit i + 1.
+ *   q [B, Hq, Nq, d]; k, v [B, Hkv, Nk, d]; o [B, Hq, Nq, d]; lse [B, Hq, Nq] or NULL.
+ *   row_kv_limit: device int32 [Nq], 4-byte aligned; values are clamped to [0, Nk].  A row with
+ *   limit 0 sees no key and gets O = 0, lse = -inf.  Key tiles past a query tile's largest
+ *   limit are skipped.  d = 64 or 128.
+ */
+int attn_fwd_prefix_masked(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                           const int32_t* row_kv_limit, float scale, int dtype, void* stream);
+
+/*
  * attn_decode - attention of Nq new query tokens per sequence against a KV cache (decoding, or
  * verifying a few drafted tokens).  "注意力即一切：从 MHA 到 GQA", section 3.4: with a KV cache the
  * keys and values of earlier tokens are stored, and each new token's query attends to all of

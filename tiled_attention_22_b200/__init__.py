@@ -13,6 +13,7 @@ from .binding import (  # noqa: F401
     ATTN_OK,
     AttnError,
     LIB_PATH,
+    apb_row_limits,
     attn_check_status,
     attn_decode,
     attn_decode_workspace_bytes,
@@ -20,6 +21,7 @@ from .binding import (  # noqa: F401
     attn_fwd,
     attn_fwd_host,
     attn_fwd_int8_quantized,
+    attn_fwd_prefix_masked,
     attn_probe_qk_int32,
     attn_quant_scratch_bytes,
     attn_quant_smooth_k,

@@ -39,6 +39,7 @@ _SIGNATURES = {
     "attn_probe_qk_int32": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp]),
     "attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i,
                            _vp, _sz, _vp]),
+    "attn_fwd_prefix_masked": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     "attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _sz, _vp]),
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "attn_check_status": (_i, []),
@@ -140,6 +141,41 @@ def attn_fwd(q, k, v, causal=False, scale=None, mode="bf16_exact", out=None, lse
                       MODES[mode], DTYPES[q.dtype], _ptr(workspace),
                       0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "attn_fwd")
+    return o, l
+
+
+def apb_row_limits(anchor: int, passing: int, local: int, device=None):
+    """Row limits of the APB layout: keys [anchor | passing | local], queries [anchor | local];
+    anchor row i sees keys < i + 1, local row i sees keys < anchor + passing + i + 1."""
+    a = torch.arange(1, anchor + 1, dtype=torch.int32)
+    l = anchor + passing + torch.arange(1, local + 1, dtype=torch.int32)
+    return torch.cat([a, l]).to(device) if device is not None else torch.cat([a, l])
+
+
+def attn_fwd_prefix_masked(q, k, v, row_kv_limit, scale=None, out=None, lse=True, stream=None):
+    """Attention where query row i sees keys j < row_kv_limit[i] (int32 CUDA tensor [Nq]).
+    q [B, Hq, Nq, d]; k, v [B, Hkv, Nk, d].  Returns (o, lse or None)."""
+    lib = load_library()
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4 or k.shape != v.shape:
+        raise ValueError("q, k, v must be [B, H, N, d] with k and v of one shape")
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if k.shape[0] != B or k.shape[3] != d:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k.shape)}")
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    if q.dtype not in DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one dtype: bfloat16 or float16")
+    if (row_kv_limit.dtype != torch.int32 or not row_kv_limit.is_cuda or row_kv_limit.numel() != Nq
+            or not row_kv_limit.is_contiguous()):
+        raise ValueError("row_kv_limit must be a contiguous int32 CUDA tensor of Nq entries")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    l = _lse_arg(lse, (B, Hq, Nq), q.device)
+    rc = lib.attn_fwd_prefix_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, Nq, Nk, d,
+                                    _ptr(row_kv_limit), scale, DTYPES[q.dtype], _stream(stream))
+    _check(rc, "attn_fwd_prefix_masked")
     return o, l
 
 

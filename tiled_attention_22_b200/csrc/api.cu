@@ -411,6 +411,18 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   return ATTN_OK;
 }
 
+int attn_fwd_prefix_masked(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                           int Nq, int Nk, int d, const int32_t* row_kv_limit, float scale, int dtype, void* stream) {
+  int rc = check_common(q, k, v, o, lse, B, Hq, Hkv, Nq, d, 0, scale, dtype);
+  if (rc) return rc;
+  if (Nk < 1 || !row_kv_limit) return ATTN_ERR_ARG;
+  if ((rc = check_shape(B, Hq, Hkv, Nk, d))) return rc;
+  if (reinterpret_cast<uintptr_t>(row_kv_limit) & 3u) return ATTN_ERR_ALIGN;
+  if (TATTN_SPLIT) return ATTN_ERR_UNSUPPORTED;  // the four-threads-per-row variant has no row limits
+  FwdParams p = make_params(B, Hq, Hkv, Nq, 0, scale, o, lse, Nk, row_kv_limit);
+  return launch_fwd<false>(q, k, v, d, dtype, p, static_cast<cudaStream_t>(stream));
+}
+
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas) {
   if (check_decode_shape(B, Hq, Hkv, Nq, Nk, d, num_ctas)) return 0;
   return decode_ws(B, Hkv, (Hq / Hkv) * Nq, decode_ctas(B, Hkv, Nk, num_ctas)).total;

@@ -39,7 +39,9 @@
 namespace tattn {
 
 struct FwdParams {
-  int B, Hq, Hkv, N, causal;
+  int B, Hq, Hkv, N, causal;  // N: query rows
+  int Nk;                 // keys (= N except under a row prefix mask)
+  const int* row_lim;     // [N] or null: query row i sees keys j < row_lim[i] (clamped to [0, Nk])
   int n_mblocks;          // ceil(N / 256)
   int sec_kv;             // kv heads per scheduling section (K/V of a section stay in L2)
   float scale_log2;       // scale * log2(e)
@@ -98,7 +100,7 @@ struct FwdCfg {
   static constexpr int OFF_BAR = OFF_V + VSTAGES * V_TILE;
   // barriers: q_full[2] k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2] o_done[2] drain
   static constexpr int NBAR = 2 + 2 * KSTAGES + 2 * VSTAGES + 6 + 1;
-  static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 16;
+  static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 32;  // + TMEM slot, abort flag, row-limit stats
   // +1024 for manual alignment of the dynamic shared memory base; at least 120 KB so that exactly
   // one CTA (which owns all 512 TMEM columns) is resident per SM.
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 120 * 1024 ? (SMEM_USED + 1024) : 120 * 1024;
@@ -286,7 +288,10 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
   }
   // exponent argument (x - off) * sc - m, off = 1.5*2^23 for INT8 (removed exactly by the add;
   // folding it into the constant would round off*sc + m per tile, shifting whole tiles)
-  const float2 sc2 = make_float2(sc, sc), cst2 = make_float2(-m_run, -m_run);
+  // (a row that has seen no key yet, possible only under a row prefix mask, keeps m = -inf: its
+  // masked scores then give exp2(-inf - 0) = 0 rather than -inf + inf)
+  const float m_use = m_run == -INFINITY ? 0.f : m_run;
+  const float2 sc2 = make_float2(sc, sc), cst2 = make_float2(-m_use, -m_use);
   const float2 off2 = make_float2(-12582912.0f, -12582912.0f);
   float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -505,15 +510,45 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
   const int mb_rank = rr / (nkv_sec * G);
   const int within = rr - mb_rank * (nkv_sec * G);
   const int kvz = kv0 + within / G;  // b * Hkv + kv head
-  const int mb = p.causal ? p.n_mblocks - 1 - mb_rank : mb_rank;
+  const int mb = (p.causal || p.row_lim) ? p.n_mblocks - 1 - mb_rank : mb_rank;
   const int b = kvz / p.Hkv;
   const int h = (kvz - b * p.Hkv) * G + within % G;
   const int bh = b * p.Hq + h;
-  const int nkv = (p.N + 127) / 128;
+  const int nkv = (p.Nk + 127) / 128;
+  // Row prefix mask: the largest and smallest limit of each query tile's rows (rows < N), from
+  // one warp, through shared memory: the largest sets the tile's key-tile count, the smallest
+  // the first key tile that needs an element mask.
+  int* lim_stats = reinterpret_cast<int*>(tmem_slot + 2);
+  if (p.row_lim != nullptr) {
+    if (warp == R::kTmaWarp) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        int mx = 0, mn = INT_MAX;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int row = mb * 256 + 128 * t + 32 * k + lane;
+          if (row < p.N) {
+            const int l = min(max(__ldg(&p.row_lim[row]), 0), p.Nk);
+            mx = max(mx, l);
+            mn = min(mn, l);
+          }
+        }
+        mx = __reduce_max_sync(0xffffffffu, mx);
+        mn = __reduce_min_sync(0xffffffffu, mn);
+        if (lane == 0) {
+          lim_stats[2 * t] = mx;
+          lim_stats[2 * t + 1] = mn;
+        }
+      }
+    }
+    __syncthreads();
+  }
   // key tiles each query tile visits (0 for a tile past N); n1 >= n0 unless tile 1 is empty
   auto key_tiles = [&](int t) {
     const int row0 = mb * 256 + 128 * t;
-    return row0 < p.N ? (p.causal ? min(nkv, row0 / 128 + 1) : nkv) : 0;
+    if (row0 >= p.N) return 0;
+    if (p.row_lim != nullptr) return (lim_stats[2 * t] + 127) / 128;
+    return p.causal ? min(nkv, row0 / 128 + 1) : nkv;
   };
   const int n0 = key_tiles(0), n1 = key_tiles(1);
   // (kept in registers: a runtime-indexed array would live in local memory)
@@ -641,13 +676,13 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nblk + j]) : sq_scale;
+        float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nkv + j]) : sq_scale;
         if constexpr (INT8) sc = fmaxf(sc, 1e-30f);
         const int col0 = j * 128;
         const bool diag = p.causal && (j == nt - 1);
-        if (diag || (col0 + 128 > p.N)) {
-          const int limA = (diag ? min(rowA + 1, p.N) : p.N) - col0;
-          const int limB = (diag ? min(rowB + 1, p.N) : p.N) - col0;
+        if (diag || (col0 + 128 > p.Nk)) {
+          const int limA = (diag ? min(rowA + 1, p.Nk) : p.Nk) - col0;
+          const int limB = (diag ? min(rowB + 1, p.Nk) : p.Nk) - col0;
           ok = softmax_step_split<D, INT8, FP16, true>(tS, tO, sc, limA, limB, j, m_run, l_run, &o_done[t],
                                                        abort_flag);
         } else {
@@ -725,20 +760,24 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       // (an empty tile, row0 >= N, reads nothing: its sq entry does not exist)
       const float sq_scale = (INT8 && nt > 0) ? p.sq[(size_t)bh * nblk + row0 / 128] * p.scale_log2 : p.scale_log2;
       float m_run = -INFINITY, l_run = 0.f;
+      // row prefix mask: this row's limit, and the tile-wide smallest limit (rows < N)
+      const int row_lim = (p.row_lim != nullptr && row < p.N) ? min(max(__ldg(&p.row_lim[row]), 0), p.Nk) : 0;
+      const int tile_min_lim = p.row_lim != nullptr ? lim_stats[2 * t + 1] : INT_MAX;
       bool ok = true;
       for (int j = 0; j < nt; ++j) {
         ok = mbar_wait(&s_full[t], j & 1, abort_flag, W_SOFTMAX + 1);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nblk + j]) : sq_scale;
+        float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nkv + j]) : sq_scale;
         if constexpr (INT8) sc = fmaxf(sc, 1e-30f);  // a zero block: keep -inf * sc = -inf for masks
-        // causal diagonal tile (key > query) and the ragged last key tile (key >= N) are masked;
-        // keys [0, lim) of the tile are visible
+        // causal diagonal tile (key > query), the ragged last key tile (key >= Nk) and, under a
+        // row prefix mask, every tile that reaches past some row's limit are masked; keys
+        // [0, lim) of the tile are visible
         const int col0 = j * 128;
         const bool diag = p.causal && (j == nt - 1);
-        if (diag || (col0 + 128 > p.N)) {
-          const int lim = (diag ? min(row + 1, p.N) : p.N) - col0;
+        if (diag || (col0 + 128 > p.Nk) || (col0 + 128 > tile_min_lim)) {
+          const int lim = (p.row_lim != nullptr ? row_lim : (diag ? min(row + 1, p.Nk) : p.Nk)) - col0;
           ok = softmax_step<D, INT8, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
         } else {
           ok = softmax_step<D, INT8, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
@@ -755,12 +794,20 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
           mbar_arrive(&p_full[t]);
         }
       }
+      if (ok && nt == 0 && p.row_lim != nullptr && row < p.N) {
+        // every row of this tile sees no key: O = 0, lse = -inf
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.o) + ((size_t)bh * p.N + row) * (D * 2));
+#pragma unroll
+        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+        if (p.lse != nullptr) p.lse[(size_t)bh * p.N + row] = -INFINITY;
+      }
       if (ok && nt > 0) {
         ok = mbar_wait(&o_done[t], 0, abort_flag, W_SOFTMAX + 3);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
           tc_fence_after();
-          const float inv_l = 1.0f / l_run;
+          // (a row that saw no key, possible only under a row prefix mask, has l = 0: O = 0)
+          const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
           uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)bh * p.N + (size_t)row) * (D * 2);
   #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -778,7 +825,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
             }
           }
           if (p.lse != nullptr && row < p.N) {
-            float lse = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+            float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
             if constexpr (INT8) lse += p.bias[(size_t)bh * p.N + row];
             p.lse[(size_t)bh * p.N + row] = lse;
           }

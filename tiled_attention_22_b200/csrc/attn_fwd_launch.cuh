@@ -17,8 +17,8 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
   const CUtensorMapDataType v_dt = FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   int rc;
   if ((rc = make_map(&tq, q, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hq, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
-  if ((rc = make_map(&tk, k, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hkv, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
-  if ((rc = make_map(&tv, v, v_dt, 2, D, p.N, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  if ((rc = make_map(&tk, k, qk_dt, C::QK_ELEM, D, p.Nk, p.B * p.Hkv, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
+  if ((rc = make_map(&tv, v, v_dt, 2, D, p.Nk, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
   auto kern = attn_fwd_kernel<D, INT8, FP16, SPLIT>;
   // Once per device: allow the dynamic shared memory, and check the register split.  The kernel
   // moves registers between warpgroups with setmaxnreg; the increase only completes if the
@@ -54,12 +54,15 @@ int launch_fwd(const void* q, const void* k, const void* v, int d, int dtype, co
   return fp16 ? launch_fwd_t<64, INT8, true>(q, k, v, p, stream) : launch_fwd_t<64, INT8, false>(q, k, v, p, stream);
 }
 
-FwdParams make_params(int B, int Hq, int Hkv, int N, int causal, float scale, void* o, float* lse) {
+FwdParams make_params(int B, int Hq, int Hkv, int N, int causal, float scale, void* o, float* lse, int Nk = -1,
+                      const int* row_lim = nullptr) {
   FwdParams p{};
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.N = N;
+  p.Nk = Nk < 0 ? N : Nk;
+  p.row_lim = row_lim;
   p.causal = causal;
   p.n_mblocks = (N + 255) / 256;
   // Scheduling sections: kv heads whose K and V (16-bit, d=128, the larger case) take at most
@@ -67,7 +70,7 @@ FwdParams make_params(int B, int Hq, int Hkv, int N, int causal, float scale, vo
 #ifndef TATTN_L2_SECTION_MB
 #define TATTN_L2_SECTION_MB 32
 #endif
-  const long long kv_bytes = 2LL * N * 128 * 2;
+  const long long kv_bytes = 2LL * p.Nk * 128 * 2;
   long long sec = ((long long)TATTN_L2_SECTION_MB << 20) / (kv_bytes > 0 ? kv_bytes : 1);
   if (sec < 1) sec = 1;
   if (sec > (long long)B * Hkv) sec = (long long)B * Hkv;
