@@ -10,6 +10,9 @@ Contents
   exact            O1: plain float64 softmax attention (the definition), also
                    with Nq < Nk (queries after a KV cache) and with a per-row
                    visible key prefix (the APB mask shape).
+  fp8_emulation    O3: the same smoothing with per-block FP8 (E4M3) codes
+                   (round to nearest even, saturating at 448) and exact
+                   code-product scores.
   int8_emulation   O2: bit-exact emulation of K smoothing and per-block INT8
                    quantisation of Q and K, exact integer QK^T, and the
                    float64 attention that follows from those quantised scores.
