@@ -275,6 +275,7 @@ def run_native(args, w, world, rank, local):
                kmean=torch.empty((B, Hkv, d), device=dev, dtype=torch.float32),
                lse_bias=torch.empty((B, Hq, N), device=dev, dtype=torch.float32))
     scratch = torch.empty(ta.attn_quant_scratch_bytes(B, Hkv, N, d), device=dev, dtype=torch.uint8)
+    pre8 = dict(pre, q8=pre["q8"].view(torch.uint8), k8=pre["k8"].view(torch.uint8))
     stream = torch.cuda.current_stream()
     flops = w.flops()
 
@@ -285,6 +286,16 @@ def run_native(args, w, world, rank, local):
         if ev:
             ev[1].record(stream)
         ta.attn_fwd_int8_quantized(pre, vd, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    def step_fp8(ev=None):
+        if ev:
+            ev[0].record(stream)
+        ta.attn_quant_smooth_k_fp8(qd, kd, scale=w.scale, scratch=scratch, stream=stream, out=pre8)
+        if ev:
+            ev[1].record(stream)
+        ta.attn_fwd_fp8_quantized(pre8, vd, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
         if ev:
             ev[2].record(stream)
 
@@ -300,7 +311,7 @@ def run_native(args, w, world, rank, local):
                            if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local)
     sampler.start()
     time.sleep(0.3)
-    for mode, fn, nk in (("int8_qk", step_int8, 2), ("bf16_exact", step_bf16, 1)):
+    for mode, fn, nk in (("int8_qk", step_int8, 2), ("bf16_exact", step_bf16, 1), ("fp8_qk", step_fp8, 2)):
         if mode not in args.modes.split(","):
             continue
         for _ in range(args.warmup):
@@ -359,6 +370,7 @@ def run_native(args, w, world, rank, local):
            "kernel_ms": [float("nan"), float("nan")]}
     r8 = results.get("int8_qk", nan)
     rb = results.get("bf16_exact", nan)
+    rf = results.get("fp8_qk", nan)
     long_region = r8["ms_total"] > 1000.0
     bf16_peak = peaks["bf16_sustained"] if long_region else peaks["bf16"]
     mixed_peak = bf16_peak * 4.0 / 3.0  # QK^T at the INT8 rate (2x bf16, nominal ratio), PV at the bf16 rate
@@ -377,6 +389,10 @@ def run_native(args, w, world, rank, local):
                         "prepass_ms": r8["kernel_ms"][0], "fused_ms": fused_ms,
                         "fused_tflops": achieved,
                         "prepass_gbs": _prepass_bytes(w) / (r8["kernel_ms"][0] * 1e-3) / 1e9},
+            "fp8_qk": {"tflops": rf["tflops"], "ms_per_step": rf["ms_per_step"],
+                       "prepass_ms": rf["kernel_ms"][0], "fused_ms": rf["kernel_ms"][1],
+                       "fused_tflops": flops / (rf["kernel_ms"][1] * 1e-3) / 1e12,
+                       "frac_of_mixed_peak": (flops / (rf["kernel_ms"][1] * 1e-3) / 1e12) / mixed_peak},
             "bf16_exact": {"tflops": rb["tflops"], "ms_per_step": rb["ms_per_step"],
                            "frac_of_bf16_peak": (flops / (rb["kernel_ms"][0] * 1e-3) / 1e12) / bf16_peak,
                            "traffic": _measured_traffic("bf16_exact"),
@@ -516,7 +532,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurements")
-    ap.add_argument("--modes", default="int8_qk,bf16_exact",
+    ap.add_argument("--modes", default="int8_qk,bf16_exact,fp8_qk",
                     help="modes to time (the headline value is int8_qk; drop one only for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:

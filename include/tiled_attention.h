@@ -59,7 +59,7 @@ enum attn_status {
   ATTN_ERR_TIMEOUT = -6       /* a device-side wait ran out (reported by attn_check_status) */
 };
 
-enum attn_mode { ATTN_MODE_BF16_EXACT = 0, ATTN_MODE_INT8_QK = 1 };
+enum attn_mode { ATTN_MODE_BF16_EXACT = 0, ATTN_MODE_INT8_QK = 1, ATTN_MODE_FP8_QK = 2 };
 enum attn_dtype { ATTN_BF16 = 0, ATTN_FP16 = 1 };
 
 /*
@@ -73,8 +73,10 @@ enum attn_dtype { ATTN_BF16 = 0, ATTN_FP16 = 1 };
  *   causal: 0 or 1 (key j is visible to query i when j <= i).
  *   scale: the softmax scale (finite, > 0), normally 1/sqrt(d).
  *   mode: ATTN_MODE_BF16_EXACT (16-bit Q K^T on tensor cores, fp32
- *     accumulation) or ATTN_MODE_INT8_QK (runs the pre-pass of
- *     attn_quant_smooth_k into `workspace`, then INT8 Q K^T).
+ *     accumulation), ATTN_MODE_INT8_QK (runs the pre-pass of
+ *     attn_quant_smooth_k into `workspace`, then INT8 Q K^T) or
+ *     ATTN_MODE_FP8_QK (the pre-pass of attn_quant_smooth_k_fp8, then FP8
+ *     E4M3 Q K^T with fp32 accumulation; same workspace size as INT8).
  *   workspace / ws_bytes: device memory of at least
  *     attn_workspace_bytes(B,Hq,Hkv,N,d,mode) bytes (0 for BF16_EXACT, where
  *     workspace may be NULL).  Its content on entry does not matter.
@@ -83,7 +85,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int d, int causal, float scale, int mode,
              int dtype, void* workspace, size_t ws_bytes, void* stream);
 
-/* Bytes of workspace attn_fwd needs for these sizes and mode (0 for BF16_EXACT). */
+/* Bytes of workspace attn_fwd needs for these sizes and mode (0 for BF16_EXACT; the 8-bit modes
+ * need the same). */
 size_t attn_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int mode);
 
 /*
@@ -113,6 +116,33 @@ int attn_quant_smooth_k(const void* q, const void* k, int B, int Hq, int Hkv, in
 
 /* Bytes of scratch attn_quant_smooth_k needs: B*Hkv*ceil(N/128)*d*8 (+ alignment). */
 size_t attn_quant_scratch_bytes(int B, int Hkv, int N, int d);
+
+/*
+ * attn_quant_smooth_k_fp8 - the pre-pass of ATTN_MODE_FP8_QK: the same K mean, smoothing and lse
+ * bias as attn_quant_smooth_k, with FP8 E4M3 codes in place of INT8 ones.  The SageAttention
+ * article (section 技术方案) weighs INT8 against FP8 for the 8-bit Q K^T; the FP8 variant keeps
+ * its smoothing and per-block scales:
+ *   per 128-token block (all d channels) amax = max|x|, scale = amax/448 (448 = largest finite
+ *   E4M3), code = E4M3(fl32(x * (448/amax))), rounded to nearest with ties to even and
+ *   saturated at +-448; an all-zero block has scale 0 and codes 0.
+ *   q8 [B,Hq,N,d], k8 [B,Hkv,N,d]: E4M3 bit patterns (1 sign, 4 exponent bits with bias 7,
+ *   3 mantissa bits, no infinities).  Other arguments as for attn_quant_smooth_k (same
+ *   scratch size).
+ */
+int attn_quant_smooth_k_fp8(const void* q, const void* k, int B, int Hq, int Hkv, int N, int d,
+                            int dtype, float scale, uint8_t* q8, float* sq, uint8_t* k8, float* sk,
+                            float* kmean, float* lse_bias, void* scratch, size_t scratch_bytes,
+                            void* stream);
+
+/*
+ * attn_fwd_fp8_quantized - the fused FP8 attention kernel alone, on the outputs of
+ * attn_quant_smooth_k_fp8: S = E4M3 Q K^T with fp32 accumulation (tcgen05.mma kind::f8f6f4),
+ * dequantised by sq * sk, online softmax, 16-bit P V.  Arguments as attn_fwd_int8_quantized.
+ */
+int attn_fwd_fp8_quantized(const uint8_t* q8, const float* sq, const uint8_t* k8,
+                           const float* sk, const float* lse_bias, const void* v, void* o,
+                           float* lse, int B, int Hq, int Hkv, int N, int d, int causal,
+                           float scale, int dtype, void* stream);
 
 /*
  * attn_quant_smooth_k_noalloc - the same pre-pass as attn_quant_smooth_k, for callers that cannot

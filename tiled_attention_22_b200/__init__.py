@@ -1,4 +1,5 @@
-"""B200 (sm_100a) tiled attention forward: bf16_exact and SageAttention-style int8_qk.
+"""B200 (sm_100a) tiled attention forward: bf16_exact, SageAttention-style int8_qk and fp8_qk,
+a row-prefix-masked variant (the APB mask shape) and a KV-cache decode path.
 
 The computation runs in the CUDA library built from ``csrc/`` (C ABI in
 ``include/tiled_attention.h``); this package only marshals arguments.
@@ -20,11 +21,13 @@ from .binding import (  # noqa: F401
     attn_error_string,
     attn_fwd,
     attn_fwd_host,
+    attn_fwd_fp8_quantized,
     attn_fwd_int8_quantized,
     attn_fwd_prefix_masked,
     attn_probe_qk_int32,
     attn_quant_scratch_bytes,
     attn_quant_smooth_k,
+    attn_quant_smooth_k_fp8,
     attn_quant_smooth_k_noalloc,
     attn_test_exp2,
     attn_test_wait_timeout,

@@ -25,7 +25,7 @@ ATTN_ERR_WORKSPACE = -4
 ATTN_ERR_LAUNCH = -5
 ATTN_ERR_TIMEOUT = -6
 
-MODES = {"bf16_exact": 0, "int8_qk": 1}
+MODES = {"bf16_exact": 0, "int8_qk": 1, "fp8_qk": 2}
 DTYPES = {torch.bfloat16: 0, torch.float16: 1}
 
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -34,6 +34,8 @@ _SIGNATURES = {
     "attn_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_quant_smooth_k": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "attn_quant_scratch_bytes": (_sz, [_i, _i, _i, _i]),
+    "attn_quant_smooth_k_fp8": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "attn_fwd_fp8_quantized": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_quant_smooth_k_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "attn_fwd_int8_quantized": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_probe_qk_int32": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp]),
@@ -282,6 +284,49 @@ def attn_fwd_int8_quantized(pre, v, causal=False, scale=None, out=None, lse=True
                                      _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, int(bool(causal)), scale,
                                      DTYPES[v.dtype], _stream(stream))
     _check(rc, "attn_fwd_int8_quantized")
+    return o, l
+
+
+def attn_quant_smooth_k_fp8(q, k, scale=None, scratch=None, stream=None, out=None):
+    """The FP8 pre-pass alone: E4M3 codes (uint8 bit patterns) and per-block scales.  Returns
+    dict(q8, sq, k8, sk, kmean, lse_bias) (``out`` if given)."""
+    lib = load_library()
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    _shape(q, k, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    T = (N + 127) // 128
+    dev = q.device
+    out = out or dict(
+        q8=torch.empty((B, Hq, N, d), device=dev, dtype=torch.uint8),
+        sq=torch.empty((B, Hq, T), device=dev, dtype=torch.float32),
+        k8=torch.empty((B, Hkv, N, d), device=dev, dtype=torch.uint8),
+        sk=torch.empty((B, Hkv, T), device=dev, dtype=torch.float32),
+        kmean=torch.empty((B, Hkv, d), device=dev, dtype=torch.float32),
+        lse_bias=torch.empty((B, Hq, N), device=dev, dtype=torch.float32),
+    )
+    if scratch is None:
+        scratch = torch.empty(attn_quant_scratch_bytes(B, Hkv, N, d), device=dev, dtype=torch.uint8)
+    rc = lib.attn_quant_smooth_k_fp8(_ptr(q), _ptr(k), B, Hq, Hkv, N, d, DTYPES[q.dtype], scale, _ptr(out["q8"]),
+                                     _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]), _ptr(out["kmean"]),
+                                     _ptr(out["lse_bias"]), _ptr(scratch), scratch.numel(), _stream(stream))
+    _check(rc, "attn_quant_smooth_k_fp8")
+    return out
+
+
+def attn_fwd_fp8_quantized(pre, v, causal=False, scale=None, out=None, lse=True, stream=None):
+    """The fused FP8 kernel on the outputs of attn_quant_smooth_k_fp8 (``pre``)."""
+    lib = load_library()
+    q8, k8 = pre["q8"], pre["k8"]
+    B, Hq, N, d = q8.shape
+    Hkv = k8.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty((B, Hq, N, d), device=v.device, dtype=v.dtype) if out is None else out
+    l = _lse_arg(lse, (B, Hq, N), v.device)
+    rc = lib.attn_fwd_fp8_quantized(_ptr(q8), _ptr(pre["sq"]), _ptr(k8), _ptr(pre["sk"]), _ptr(pre["lse_bias"]),
+                                    _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, int(bool(causal)), scale,
+                                    DTYPES[v.dtype], _stream(stream))
+    _check(rc, "attn_fwd_fp8_quantized")
     return o, l
 
 

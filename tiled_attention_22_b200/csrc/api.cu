@@ -92,9 +92,30 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int N, int d) {
   return w;
 }
 
+template <bool F8>
+int launch_quant(const uint16_t* q16, const uint16_t* k16, int B, int Hq, int Hkv, int N, int d, bool fp16,
+                 float scale, const float* kmean, int8_t* q8, float* sq, int8_t* k8, float* sk, float* bias,
+                 unsigned qblocks, cudaStream_t stream) {
+  if (d == 128) {
+    if (fp16)
+      quant_kernel<128, true, F8><<<qblocks, quant_threads<128>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+    else
+      quant_kernel<128, false, F8><<<qblocks, quant_threads<128>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+  } else {
+    if (fp16)
+      quant_kernel<64, true, F8><<<qblocks, quant_threads<64>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+    else
+      quant_kernel<64, false, F8><<<qblocks, quant_threads<64>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
+  }
+  TATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
+}
+
+// The pre-pass: K channel mean (float64 partials, then the final division), then smoothing and
+// quantisation of K and quantisation of Q with the lse bias; f8 selects E4M3 codes over INT8.
 int launch_prepass(const void* q, const void* k, int B, int Hq, int Hkv, int N, int d, int dtype, float scale,
                    int8_t* q8, float* sq, int8_t* k8, float* sk, float* kmean, float* bias, double* part,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, bool f8 = false) {
   const int T = (N + 127) / 128;
   const int BG = B * Hkv;
   const bool fp16 = dtype == ATTN_FP16;
@@ -114,29 +135,18 @@ int launch_prepass(const void* q, const void* k, int B, int Hq, int Hkv, int N, 
   kmean_final_kernel<<<(BG * d + 127) / 128, 128, 0, stream>>>(part, BG, N, d, kmean);
   TATTN_CUDA(cudaGetLastError());
   const unsigned qblocks = (unsigned)((long long)B * Hkv * T + (long long)B * Hq * T);
-  if (d == 128) {
-    if (fp16)
-      quant_kernel<128, true><<<qblocks, quant_threads<128>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
-    else
-      quant_kernel<128, false><<<qblocks, quant_threads<128>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
-  } else {
-    if (fp16)
-      quant_kernel<64, true><<<qblocks, quant_threads<64>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
-    else
-      quant_kernel<64, false><<<qblocks, quant_threads<64>(), 0, stream>>>(q16, k16, B, Hq, Hkv, N, scale, kmean, q8, sq, k8, sk, bias);
-  }
-  TATTN_CUDA(cudaGetLastError());
-  return ATTN_OK;
+  return f8 ? launch_quant<true>(q16, k16, B, Hq, Hkv, N, d, fp16, scale, kmean, q8, sq, k8, sk, bias, qblocks, stream)
+            : launch_quant<false>(q16, k16, B, Hq, Hkv, N, d, fp16, scale, kmean, q8, sq, k8, sk, bias, qblocks, stream);
 }
 
-int fwd_int8_quantized(const int8_t* q8, const float* sq, const int8_t* k8, const float* sk, const float* bias,
-                       const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal,
-                       float scale, int dtype, cudaStream_t stream) {
+int fwd_quantized(const void* q8, const float* sq, const void* k8, const float* sk, const float* bias, const void* v,
+                  void* o, float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, int dtype,
+                  bool f8, cudaStream_t stream) {
   FwdParams p = make_params(B, Hq, Hkv, N, causal, scale, o, lse);
   p.sq = sq;
   p.sk = sk;
   p.bias = bias;
-  return launch_fwd<true>(q8, k8, v, d, dtype, p, stream);
+  return f8 ? launch_fwd<QK_F8>(q8, k8, v, d, dtype, p, stream) : launch_fwd<QK_I8>(q8, k8, v, d, dtype, p, stream);
 }
 
 __global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int use_poly) {
@@ -205,7 +215,7 @@ int static_scratch_address(double** out) {
 extern "C" {
 
 size_t attn_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int mode) {
-  if (mode != ATTN_MODE_INT8_QK) return 0;
+  if (mode != ATTN_MODE_INT8_QK && mode != ATTN_MODE_FP8_QK) return 0;
   if (check_shape(B, Hq, Hkv, N, d)) return 0;
   return ws_layout(B, Hq, Hkv, N, d).total;
 }
@@ -264,8 +274,36 @@ int attn_fwd_int8_quantized(const int8_t* q8, const float* sq, const int8_t* k8,
   int rc = check_common(q8, k8, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype);
   if (rc) return rc;
   if (!sq || !sk || (lse && !lse_bias)) return ATTN_ERR_ARG;
-  return fwd_int8_quantized(q8, sq, k8, sk, lse_bias, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype,
-                            static_cast<cudaStream_t>(stream));
+  return fwd_quantized(q8, sq, k8, sk, lse_bias, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype, false,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int attn_quant_smooth_k_fp8(const void* q, const void* k, int B, int Hq, int Hkv, int N, int d, int dtype,
+                            float scale, uint8_t* q8, float* sq, uint8_t* k8, float* sk, float* kmean,
+                            float* lse_bias, void* scratch, size_t scratch_bytes_given, void* stream) {
+  if (!q || !k || !q8 || !sq || !k8 || !sk || !kmean || !lse_bias) return ATTN_ERR_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_ARG;
+  int rc = check_shape(B, Hq, Hkv, N, d);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q8) || !aligned16(k8) || !aligned16(kmean) || !aligned16(sq) ||
+      !aligned16(sk) || !aligned16(lse_bias))
+    return ATTN_ERR_ALIGN;
+  if (!scratch || scratch_bytes_given < scratch_bytes(B, Hkv, N, d)) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(scratch)) return ATTN_ERR_ALIGN;
+  return launch_prepass(q, k, B, Hq, Hkv, N, d, dtype, scale, reinterpret_cast<int8_t*>(q8), sq,
+                        reinterpret_cast<int8_t*>(k8), sk, kmean, lse_bias, static_cast<double*>(scratch),
+                        static_cast<cudaStream_t>(stream), true);
+}
+
+int attn_fwd_fp8_quantized(const uint8_t* q8, const float* sq, const uint8_t* k8, const float* sk,
+                           const float* lse_bias, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                           int d, int causal, float scale, int dtype, void* stream) {
+  int rc = check_common(q8, k8, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype);
+  if (rc) return rc;
+  if (!sq || !sk || (lse && !lse_bias)) return ATTN_ERR_ARG;
+  return fwd_quantized(q8, sq, k8, sk, lse_bias, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype, true,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N, int d,
@@ -275,9 +313,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mode == ATTN_MODE_BF16_EXACT) {
     FwdParams p = make_params(B, Hq, Hkv, N, causal, scale, o, lse);
-    return launch_fwd<false>(q, k, v, d, dtype, p, st);
+    return launch_fwd<QK_F16>(q, k, v, d, dtype, p, st);
   }
-  if (mode != ATTN_MODE_INT8_QK) return ATTN_ERR_ARG;
+  if (mode != ATTN_MODE_INT8_QK && mode != ATTN_MODE_FP8_QK) return ATTN_ERR_ARG;
+  const bool f8 = mode == ATTN_MODE_FP8_QK;
   const WsLayout w = ws_layout(B, Hq, Hkv, N, d);
   if (!workspace || ws_bytes < w.total) return ATTN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
@@ -289,9 +328,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   auto* kmean = reinterpret_cast<float*>(ws + w.kmean);
   auto* bias = reinterpret_cast<float*>(ws + w.bias);
   auto* part = reinterpret_cast<double*>(ws + w.scratch);
-  rc = launch_prepass(q, k, B, Hq, Hkv, N, d, dtype, scale, q8, sq, k8, sk, kmean, bias, part, st);
+  rc = launch_prepass(q, k, B, Hq, Hkv, N, d, dtype, scale, q8, sq, k8, sk, kmean, bias, part, st, f8);
   if (rc) return rc;
-  return fwd_int8_quantized(q8, sq, k8, sk, bias, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype, st);
+  return fwd_quantized(q8, sq, k8, sk, bias, v, o, lse, B, Hq, Hkv, N, d, causal, scale, dtype, f8, st);
 }
 
 int attn_probe_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int Hkv, int N, int d,
@@ -322,7 +361,8 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   if (!q || !k || !v || !o) return ATTN_ERR_ARG;
   int rc = check_common(dq, dk, dv, do_, dlse, B, Hq, Hkv, N, d, causal, scale, dtype);
   if (rc) return rc;
-  if (mode == ATTN_MODE_INT8_QK && (!workspace || ws_bytes < attn_workspace_bytes(B, Hq, Hkv, N, d, mode)))
+  if (mode != ATTN_MODE_BF16_EXACT && mode != ATTN_MODE_INT8_QK && mode != ATTN_MODE_FP8_QK) return ATTN_ERR_ARG;
+  if (mode != ATTN_MODE_BF16_EXACT && (!workspace || ws_bytes < attn_workspace_bytes(B, Hq, Hkv, N, d, mode)))
     return ATTN_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool want_lse = lse && dlse;
@@ -420,7 +460,7 @@ int attn_fwd_prefix_masked(const void* q, const void* k, const void* v, void* o,
   if (reinterpret_cast<uintptr_t>(row_kv_limit) & 3u) return ATTN_ERR_ALIGN;
   if (TATTN_SPLIT) return ATTN_ERR_UNSUPPORTED;  // the four-threads-per-row variant has no row limits
   FwdParams p = make_params(B, Hq, Hkv, Nq, 0, scale, o, lse, Nk, row_kv_limit);
-  return launch_fwd<false>(q, k, v, d, dtype, p, static_cast<cudaStream_t>(stream));
+  return launch_fwd<QK_F16>(q, k, v, d, dtype, p, static_cast<cudaStream_t>(stream));
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_ctas) {

@@ -8,7 +8,8 @@
 // through shared memory, a running row maximum m and row sum l rescale the partial output, and the
 // N x N scores exist only as 128 x 128 tiles in tensor memory.  In INT8 mode the Q K^T tile is an
 // INT8 x INT8 -> int32 product of the pre-pass outputs, dequantised by sq * sk (SageAttention
-// article, section 技术方案), and P V stays in 16-bit floating point.
+// article, section 技术方案), and P V stays in 16-bit floating point.  FP8 mode is the same with
+// E4M3 codes and an fp32 product (tcgen05.mma kind::f8f6f4).
 //
 // B200 design (not the pages'; their kernels target Ampere/Ada/Hopper):
 //   * CTA = 2 query tiles of 128 rows, 384 threads in four roles:
@@ -47,15 +48,16 @@ struct FwdParams {
   float scale_log2;       // scale * log2(e)
   void* o;                // [B, Hq, N, D] 16-bit
   float* lse;             // [B, Hq, N] or null
-  const float* sq;        // INT8: [B, Hq, ceil(N/128)]
-  const float* sk;        // INT8: [B, Hkv, ceil(N/128)]
-  const float* bias;      // INT8: [B, Hq, N] (null allowed when lse is null)
+  const float* sq;        // 8-bit modes: [B, Hq, ceil(N/128)]
+  const float* sk;        // 8-bit modes: [B, Hkv, ceil(N/128)]
+  const float* bias;      // 8-bit modes: [B, Hq, N] (null allowed when lse is null)
 };
 
-template <int D, bool INT8>
+// BYTE: Q and K staged as 1-byte codes (INT8 or FP8 modes), else 16-bit.
+template <int D, bool BYTE>
 struct FwdCfg {
   static constexpr int BM = 128, BN = 128, QT = 2;
-  static constexpr int QK_ELEM = INT8 ? 1 : 2;                 // bytes per Q/K element
+  static constexpr int QK_ELEM = BYTE ? 1 : 2;                 // bytes per Q/K element
   static constexpr int QK_ROW = D * QK_ELEM;                   // bytes per Q/K row
   static constexpr int QK_SPAN = QK_ROW >= 128 ? 128 : 64;     // swizzle span (bytes)
   static constexpr uint32_t QK_SWZ = QK_SPAN == 128 ? kSwizzle128B : kSwizzle64B;
@@ -92,8 +94,8 @@ struct FwdCfg {
 #ifndef TATTN_VS_128I
 #define TATTN_VS_128I 3
 #endif
-  static constexpr int KSTAGES = D == 128 ? (INT8 ? TATTN_KS_128I : TATTN_KS_128B) : 4;
-  static constexpr int VSTAGES = D == 128 ? (INT8 ? TATTN_VS_128I : TATTN_VS_128B) : 4;
+  static constexpr int KSTAGES = D == 128 ? (BYTE ? TATTN_KS_128I : TATTN_KS_128B) : 4;
+  static constexpr int VSTAGES = D == 128 ? (BYTE ? TATTN_VS_128I : TATTN_VS_128B) : 4;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QT * Q_TILE;
   static constexpr int OFF_V = OFF_K + KSTAGES * K_TILE;
@@ -146,10 +148,17 @@ struct FwdRoles {
 enum : int { W_LOAD = 0x10, W_MMA = 0x20, W_SOFTMAX = 0x30, W_DRAIN = 0x40, W_PROBE = 0x50 };
 
 // Issue the QK_STEPS MMAs of S(tmem) = Q_tile * K_tile^T; both operands K-major, swizzled.
-template <int D, bool INT8, bool FP16>
+// Kind of the Q K^T product: 16-bit inputs (fp32 accumulate), INT8 codes (int32 accumulate) or
+// FP8 E4M3 codes (fp32 accumulate).  The two 8-bit kinds share the 1-byte staging layout.
+enum : int { QK_F16 = 0, QK_I8 = 1, QK_F8 = 2 };
+
+template <int D, int QK, bool FP16>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint32_t k_smem) {
-  using C = FwdCfg<D, INT8>;
-  constexpr uint32_t idesc = INT8 ? instr_desc(2, 1, 0, 0, 128, 128) : instr_desc(1, FP16 ? 0 : 1, 0, 0, 128, 128);
+  constexpr bool INT8 = QK == QK_I8;
+  using C = FwdCfg<D, QK != QK_F16>;
+  constexpr uint32_t idesc = INT8             ? instr_desc(2, 1, 0, 0, 128, 128)
+                             : QK == QK_F8 ? instr_desc(1, 0, 0, 0, 128, 128)  // E4M3 x E4M3 -> F32
+                                           : instr_desc(1, FP16 ? 0 : 1, 0, 0, 128, 128);
 #pragma unroll
   for (int kk = 0; kk < C::QK_STEPS; ++kk) {
     const uint32_t off = (uint32_t)((kk * 32) / C::QK_SPAN) * C::QK_PANEL_BYTES + (uint32_t)((kk * 32) % C::QK_SPAN);
@@ -157,6 +166,8 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint3
     const uint64_t bd = smem_desc(k_smem + off, 16, 8 * C::QK_SPAN, C::QK_SWZ);
     if constexpr (INT8)
       mma_i8_ss(s_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+    else if constexpr (QK == QK_F8)
+      mma_f8_ss(s_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
     else
       mma_f16_ss(s_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
   }
@@ -247,10 +258,11 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
-template <int D, bool INT8, bool FP16, bool MASKED>
+template <int D, int QK, bool FP16, bool MASKED>
 __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc, int lim, int j, float& m_run,
                                              float& l_run, uint64_t* o_done_t, volatile int* abort_flag) {
-  using C = FwdCfg<D, INT8>;
+  constexpr bool INT8 = QK == QK_I8;  // int32 scores (the FP8 kind's are fp32 like the 16-bit one's)
+  using C = FwdCfg<D, QK != QK_F16>;
   uint32_t r[4][32];
 #pragma unroll
   for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
@@ -344,10 +356,11 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
 // reduced over the 4 threads of a row with two xor-shuffles; each thread keeps a partial row sum
 // (summed over the 4 threads in the epilogue).  P goes back with a 16x128b store, which puts the
 // packed pair of columns (8k + 2(t%4), +1) at packed column 4k + t%4 of the same rows.
-template <int D, bool INT8, bool FP16, bool MASKED>
+template <int D, int QK, bool FP16, bool MASKED>
 __device__ __forceinline__ bool softmax_step_split(uint32_t tS, uint32_t tO, float sc, int limA, int limB, int j,
                                                    float (&m_run)[2], float (&l_run)[2], uint64_t* o_done_t,
                                                    volatile int* abort_flag) {
+  constexpr bool INT8 = QK == QK_I8;
   const int q4 = threadIdx.x & 3;
   uint32_t r[64];
   tmem_ld_16x256_x16(tS, r);
@@ -408,7 +421,7 @@ __device__ __forceinline__ bool softmax_step_split(uint32_t tS, uint32_t tO, flo
     const float2 a = ffma2(xa, sc2, cA);
     const float2 b = ffma2(xb, sc2, cB);
     float pa0, pa1, pb0, pb1;
-    if (!MASKED && (k & 7) >= 8 - FwdCfg<D, INT8>::POLY_PER_16 / 2) {
+    if (!MASKED && (k & 7) >= 8 - FwdCfg<D, QK != QK_F16>::POLY_PER_16 / 2) {
       pa0 = exp2_poly(a.x);
       pa1 = exp2_poly(a.y);
       pb0 = exp2_poly(b.x);
@@ -445,11 +458,12 @@ __device__ __forceinline__ bool softmax_step_split(uint32_t tS, uint32_t tO, flo
   return true;
 }
 
-template <int D, bool INT8, bool FP16, bool SPLIT>
+template <int D, int QK, bool FP16, bool SPLIT>
 __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdCfg<D, INT8>;
+  constexpr bool QUANT = QK != QK_F16;  // 8-bit codes with per-block scales sq, sk and the lse bias
+  using C = FwdCfg<D, QUANT>;
   using R = FwdRoles<SPLIT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -615,7 +629,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
           if (n_of(t) == 0) continue;
           if (!(ok = mbar_wait(&q_full[t], 0, abort_flag, W_MMA + 2))) break;
           tc_fence_after();
-          issue_qk<D, INT8, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr);
+          issue_qk<D, QK, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr);
           mma_commit(&s_full[t]);
           if (users_last(0) == t) mma_commit(&k_empty[0]);
         }
@@ -639,7 +653,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
               if (!(ok = mbar_wait(&k_full[ks1], ((j + 1) / C::KSTAGES) & 1, abort_flag, W_MMA + 5))) break;
               tc_fence_after();
             }
-            issue_qk<D, INT8, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr + ks1 * C::K_TILE);
+            issue_qk<D, QK, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr + ks1 * C::K_TILE);
             mma_commit(&s_full[t]);
             if (users_last(j + 1) == t) mma_commit(&k_empty[ks1]);
           }
@@ -668,7 +682,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       const uint32_t tO = tmem + C::tm_o(t) + ((uint32_t)lane_base << 16);
       const int nblk = (p.N + 127) / 128;
       const float sq_scale =
-          (INT8 && nt > 0) ? p.sq[(size_t)bh * nblk + row0 / 128] * p.scale_log2 : p.scale_log2;
+          (QUANT && nt > 0) ? p.sq[(size_t)bh * nblk + row0 / 128] * p.scale_log2 : p.scale_log2;
       float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
       bool ok = true;
       for (int j = 0; j < nt; ++j) {
@@ -676,17 +690,17 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nkv + j]) : sq_scale;
-        if constexpr (INT8) sc = fmaxf(sc, 1e-30f);
+        float sc = QUANT ? sq_scale * __ldg(&p.sk[(size_t)kvz * nkv + j]) : sq_scale;
+        if constexpr (QUANT) sc = fmaxf(sc, 1e-30f);
         const int col0 = j * 128;
         const bool diag = p.causal && (j == nt - 1);
         if (diag || (col0 + 128 > p.Nk)) {
           const int limA = (diag ? min(rowA + 1, p.Nk) : p.Nk) - col0;
           const int limB = (diag ? min(rowB + 1, p.Nk) : p.Nk) - col0;
-          ok = softmax_step_split<D, INT8, FP16, true>(tS, tO, sc, limA, limB, j, m_run, l_run, &o_done[t],
+          ok = softmax_step_split<D, QK, FP16, true>(tS, tO, sc, limA, limB, j, m_run, l_run, &o_done[t],
                                                        abort_flag);
         } else {
-          ok = softmax_step_split<D, INT8, FP16, false>(tS, tO, sc, 128, 128, j, m_run, l_run, &o_done[t],
+          ok = softmax_step_split<D, QK, FP16, false>(tS, tO, sc, 128, 128, j, m_run, l_run, &o_done[t],
                                                         abort_flag);
         }
         if (!ok) break;
@@ -740,7 +754,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
               const int row = h ? rowB : rowA;
               if (row < p.N) {
                 float lse = (m_run[h] + __log2f(l_run[h])) * 0.69314718055994531f;
-                if constexpr (INT8) lse += p.bias[(size_t)bh * p.N + row];
+                if constexpr (QUANT) lse += p.bias[(size_t)bh * p.N + row];
                 p.lse[(size_t)bh * p.N + row] = lse;
               }
             }
@@ -758,7 +772,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       const uint32_t tO = tmem + C::tm_o(t) + ((uint32_t)(wq * 32) << 16);
       const int nblk = (p.N + 127) / 128;
       // (an empty tile, row0 >= N, reads nothing: its sq entry does not exist)
-      const float sq_scale = (INT8 && nt > 0) ? p.sq[(size_t)bh * nblk + row0 / 128] * p.scale_log2 : p.scale_log2;
+      const float sq_scale = (QUANT && nt > 0) ? p.sq[(size_t)bh * nblk + row0 / 128] * p.scale_log2 : p.scale_log2;
       float m_run = -INFINITY, l_run = 0.f;
       // row prefix mask: this row's limit, and the tile-wide smallest limit (rows < N)
       const int row_lim = (p.row_lim != nullptr && row < p.N) ? min(max(__ldg(&p.row_lim[row]), 0), p.Nk) : 0;
@@ -769,8 +783,8 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        float sc = INT8 ? sq_scale * __ldg(&p.sk[(size_t)kvz * nkv + j]) : sq_scale;
-        if constexpr (INT8) sc = fmaxf(sc, 1e-30f);  // a zero block: keep -inf * sc = -inf for masks
+        float sc = QUANT ? sq_scale * __ldg(&p.sk[(size_t)kvz * nkv + j]) : sq_scale;
+        if constexpr (QUANT) sc = fmaxf(sc, 1e-30f);  // a zero block: keep -inf * sc = -inf for masks
         // causal diagonal tile (key > query), the ragged last key tile (key >= Nk) and, under a
         // row prefix mask, every tile that reaches past some row's limit are masked; keys
         // [0, lim) of the tile are visible
@@ -778,9 +792,9 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         const bool diag = p.causal && (j == nt - 1);
         if (diag || (col0 + 128 > p.Nk) || (col0 + 128 > tile_min_lim)) {
           const int lim = (p.row_lim != nullptr ? row_lim : (diag ? min(row + 1, p.Nk) : p.Nk)) - col0;
-          ok = softmax_step<D, INT8, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
+          ok = softmax_step<D, QK, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
         } else {
-          ok = softmax_step<D, INT8, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
+          ok = softmax_step<D, QK, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
         }
         if (!ok) break;
         tmem_st_wait();
@@ -826,7 +840,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
           }
           if (p.lse != nullptr && row < p.N) {
             float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-            if constexpr (INT8) lse += p.bias[(size_t)bh * p.N + row];
+            if constexpr (QUANT) lse += p.bias[(size_t)bh * p.N + row];
             p.lse[(size_t)bh * p.N + row] = lse;
           }
         }
@@ -898,7 +912,7 @@ __global__ void __launch_bounds__(160, 1)
       }
       if (mbar_wait(&bars[0], 0, abort_flag, W_PROBE + 1)) {
         tc_fence_after();
-        issue_qk<D, true, false>(tmem, smem_u32(sQ), smem_u32(sK));
+        issue_qk<D, QK_I8, false>(tmem, smem_u32(sQ), smem_u32(sK));
       }
       mma_commit(&bars[1]);
     }

@@ -6,20 +6,21 @@
 #define TATTN_SPLIT 0
 #endif
 
-template <int D, bool INT8, bool FP16>
+template <int D, int QK, bool FP16>
 int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p, cudaStream_t stream) {
-  using C = FwdCfg<D, INT8>;
+  constexpr bool BYTE = QK != QK_F16;
+  using C = FwdCfg<D, BYTE>;
   constexpr bool SPLIT = TATTN_SPLIT != 0;
   using R = FwdRoles<SPLIT>;
   CUtensorMap tq, tk, tv;
   const CUtensorMapDataType qk_dt =
-      INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : (FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+      BYTE ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : (FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
   const CUtensorMapDataType v_dt = FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   int rc;
   if ((rc = make_map(&tq, q, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hq, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
   if ((rc = make_map(&tk, k, qk_dt, C::QK_ELEM, D, p.Nk, p.B * p.Hkv, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
   if ((rc = make_map(&tv, v, v_dt, 2, D, p.Nk, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
-  auto kern = attn_fwd_kernel<D, INT8, FP16, SPLIT>;
+  auto kern = attn_fwd_kernel<D, QK, FP16, SPLIT>;
   // Once per device: allow the dynamic shared memory, and check the register split.  The kernel
   // moves registers between warpgroups with setmaxnreg; the increase only completes if the
   // registers the CTA is launched with cover the split, so refuse to launch otherwise.
@@ -46,12 +47,12 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
   return ATTN_OK;
 }
 
-template <bool INT8>
+template <int QK>
 int launch_fwd(const void* q, const void* k, const void* v, int d, int dtype, const FwdParams& p,
                cudaStream_t stream) {
   const bool fp16 = dtype == ATTN_FP16;
-  if (d == 128) return fp16 ? launch_fwd_t<128, INT8, true>(q, k, v, p, stream) : launch_fwd_t<128, INT8, false>(q, k, v, p, stream);
-  return fp16 ? launch_fwd_t<64, INT8, true>(q, k, v, p, stream) : launch_fwd_t<64, INT8, false>(q, k, v, p, stream);
+  if (d == 128) return fp16 ? launch_fwd_t<128, QK, true>(q, k, v, p, stream) : launch_fwd_t<128, QK, false>(q, k, v, p, stream);
+  return fp16 ? launch_fwd_t<64, QK, true>(q, k, v, p, stream) : launch_fwd_t<64, QK, false>(q, k, v, p, stream);
 }
 
 FwdParams make_params(int B, int Hq, int Hkv, int N, int causal, float scale, void* o, float* lse, int Nk = -1,

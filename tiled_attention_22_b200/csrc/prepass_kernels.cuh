@@ -101,7 +101,16 @@ __global__ void __launch_bounds__(128) kmean_final_kernel(const double* __restri
 template <int D>
 constexpr int quant_threads() { return 4 * D; }
 
-template <int D, bool FP16>
+// Two float32 values to two E4M3 codes (round to nearest even, saturating at +-448): lo in the
+// low byte, hi in the high byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// F8: FP8 (E4M3) codes with scale amax/448 instead of INT8 codes with scale amax/127.
+template <int D, bool FP16, bool F8>
 __global__ void __launch_bounds__(4 * D, 256 / D) quant_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                                                         int B, int Hq, int Hkv, int N, float scale,
                                                         const float* __restrict__ kmean, int8_t* __restrict__ q8,
@@ -177,25 +186,42 @@ __global__ void __launch_bounds__(4 * D, 256 / D) quant_kernel(const uint16_t* _
   for (int w = 1; w < NW; ++w) amax = fmaxf(amax, warp_max[w]);
 
   const bool zero = (amax == 0.f);
-  const float scl = zero ? 0.f : __fdiv_rn(amax, 127.0f);
-  const float inv = zero ? 0.f : __fdiv_rn(127.0f, amax);
+  constexpr float QMAX = F8 ? 448.0f : 127.0f;  // largest code magnitude
+  const float scl = zero ? 0.f : __fdiv_rn(amax, QMAX);
+  const float inv = zero ? 0.f : __fdiv_rn(QMAX, amax);
   if (tid == 0) (is_k ? sk : sq)[(size_t)bh * T + t] = scl;
 
-  // code = rint(fl(x * inv)): the product is rounded once (__fmul_rn), then adding 1.5 * 2^23
-  // rounds it to the nearest integer, ties to even (float32 spacing is 1 on [2^23, 2^24)), and the
-  // low byte of the sum's bit pattern is the code in two's complement.  No clamp is needed:
-  // |x| <= amax and inv <= (127/amax)(1 + 2^-24), so |fl(x * inv)| < 127.5 and |code| <= 127.
-  // (A zero block has inv = 0 and gives code 0.)
+  if constexpr (F8) {
+    // code = E4M3(fl(x * inv)); |fl(x * inv)| <= 448 (1 + 2^-23), which rounds to 448 at most
 #pragma unroll
-  for (int ps = 0; ps < PASSES; ++ps) {
-    const int row = ps * RPP + r_in;
-    if (row < cnt) {
-      uint32_t b[8];
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int row = ps * RPP + r_in;
+      if (row < cnt) {
+        uint32_t h[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) b[c] = __float_as_uint(__fadd_rn(__fmul_rn(x[ps][c], inv), 12582912.0f));
-      const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
-      const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
-      *reinterpret_cast<uint2*>(dst + (size_t)row * D + chunk * 8) = make_uint2(w0, w1);
+        for (int c = 0; c < 4; ++c)
+          h[c] = e4m3x2(__fmul_rn(x[ps][2 * c], inv), __fmul_rn(x[ps][2 * c + 1], inv));
+        *reinterpret_cast<uint2*>(dst + (size_t)row * D + chunk * 8) =
+            make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+      }
+    }
+  } else {
+    // code = rint(fl(x * inv)): the product is rounded once (__fmul_rn), then adding 1.5 * 2^23
+    // rounds it to the nearest integer, ties to even (float32 spacing is 1 on [2^23, 2^24)), and the
+    // low byte of the sum's bit pattern is the code in two's complement.  No clamp is needed:
+    // |x| <= amax and inv <= (127/amax)(1 + 2^-24), so |fl(x * inv)| < 127.5 and |code| <= 127.
+    // (A zero block has inv = 0 and gives code 0.)
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int row = ps * RPP + r_in;
+      if (row < cnt) {
+        uint32_t b[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) b[c] = __float_as_uint(__fadd_rn(__fmul_rn(x[ps][c], inv), 12582912.0f));
+        const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+        const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+        *reinterpret_cast<uint2*>(dst + (size_t)row * D + chunk * 8) = make_uint2(w0, w1);
+      }
     }
   }
 }
