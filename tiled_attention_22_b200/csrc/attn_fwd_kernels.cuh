@@ -94,14 +94,37 @@ struct FwdCfg {
 #ifndef TATTN_VS_128I
 #define TATTN_VS_128I 3
 #endif
-  static constexpr int KSTAGES = D == 128 ? (BYTE ? TATTN_KS_128I : TATTN_KS_128B) : 4;
-  static constexpr int VSTAGES = D == 128 ? (BYTE ? TATTN_VS_128I : TATTN_VS_128B) : 4;
+  // P in shared memory (compile-time alternative, 8-bit modes only, where the extra 64 KB fit): P of
+  // query tile t lives in its own 128 x 128 16-bit buffer (K-major, 128-byte swizzle, two 64-key
+  // panels) instead of over S in TMEM, so the next tile's Q K^T can overwrite S as soon as the
+  // softmax has read it.  Measured 5-12% slower than P in TMEM on the named workloads: P V then
+  // reads both operands from shared memory and the softmax writes P there, which doubles the
+  // shared-memory traffic of a tile pair (about 256 KB instead of 128 KB, more cycles at 128 B/clk
+  // than the pair's tensor work).  Off by default.
+#ifndef TATTN_PSMEM
+#define TATTN_PSMEM 0
+#endif
+  static constexpr bool PSMEM = BYTE && TATTN_PSMEM;
+#ifndef TATTN_KS_PS128
+#define TATTN_KS_PS128 3
+#endif
+#ifndef TATTN_VS_PS128
+#define TATTN_VS_PS128 2
+#endif
+  static constexpr int KSTAGES = PSMEM ? (D == 128 ? TATTN_KS_PS128 : 4)
+                                       : (D == 128 ? (BYTE ? TATTN_KS_128I : TATTN_KS_128B) : 4);
+  static constexpr int VSTAGES = PSMEM ? (D == 128 ? TATTN_VS_PS128 : 4)
+                                       : (D == 128 ? (BYTE ? TATTN_VS_128I : TATTN_VS_128B) : 4);
+  static constexpr int P_PANEL_BYTES = 128 * 128;              // 128 rows x 64 keys x 2 B
+  static constexpr int P_TILE = PSMEM ? 2 * P_PANEL_BYTES : 0;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + QT * Q_TILE;
+  static constexpr int OFF_P = OFF_Q + QT * Q_TILE;
+  static constexpr int OFF_K = OFF_P + QT * P_TILE;
   static constexpr int OFF_V = OFF_K + KSTAGES * K_TILE;
   static constexpr int OFF_BAR = OFF_V + VSTAGES * V_TILE;
-  // barriers: q_full[2] k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2] o_done[2] drain
-  static constexpr int NBAR = 2 + 2 * KSTAGES + 2 * VSTAGES + 6 + 1;
+  // barriers: q_full[2] k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2] o_done[2]
+  // drain, then (P in shared memory) s_free[2] pv_done[2]
+  static constexpr int NBAR = 2 + 2 * KSTAGES + 2 * VSTAGES + 6 + 1 + 4;
   static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 32;  // + TMEM slot, abort flag, row-limit stats
   // +1024 for manual alignment of the dynamic shared memory base; at least 120 KB so that exactly
   // one CTA (which owns all 512 TMEM columns) is resident per SM.
@@ -458,6 +481,109 @@ __device__ __forceinline__ bool softmax_step_split(uint32_t tS, uint32_t tO, flo
   return true;
 }
 
+// Issue O(tmem) (+)= P(smem, 16-bit, K-major, 128-byte swizzle, two 64-key panels) * V_tile(smem,
+// MN-major, 128-byte swizzle).
+template <int D, bool FP16>
+__device__ __forceinline__ void issue_pv_ss(uint32_t o_tmem, uint32_t p_smem, uint32_t v_smem, bool accumulate) {
+  constexpr uint32_t idesc = instr_desc(1, FP16 ? 0 : 1, 0, 1, 128, D);
+#pragma unroll
+  for (int kk = 0; kk < 128 / 16; ++kk) {
+    const uint64_t ad = smem_desc(p_smem + (kk >> 2) * (128 * 128) + (uint32_t)(kk & 3) * 32, 16, 1024, kSwizzle128B);
+    const uint64_t bd = smem_desc(v_smem + kk * 16 * 128, 128 * 128, 1024, kSwizzle128B);
+    mma_f16_ss(o_tmem, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// softmax_step with P written to shared memory (see FwdCfg::PSMEM).  After S is in registers the
+// warp arrives on s_free (the MMA issuer may overwrite S with the next tile's scores); before
+// writing P it waits for P V of the previous tile (phase j - 1 of pv_done: every tile waits for
+// the phase just before its own, so the awaited phase is never ambiguous), which also makes the
+// O rescale safe.  p_row: shared address of this thread's row in panel 0 of the P buffer.
+template <int D, int QK, bool FP16, bool MASKED>
+__device__ __forceinline__ bool softmax_step_ps(uint32_t tS, uint32_t tO, float sc, int lim, int j, float& m_run,
+                                                float& l_run, uint64_t* s_free_t, uint64_t* pv_done_t,
+                                                uint32_t p_row, uint32_t p_xor, volatile int* abort_flag) {
+  constexpr bool INT8 = QK == QK_I8;  // int32 scores
+  const int lane = threadIdx.x & 31;
+  uint32_t r[4][32];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(s_free_t);
+  float x[128];
+#pragma unroll
+  for (int i = 0; i < 128; ++i) {
+    const uint32_t bits = r[i >> 5][i & 31];
+    x[i] = INT8 ? __uint_as_float(bits + 0x4B400000u) : __uint_as_float(bits);
+    if (MASKED && i >= lim) x[i] = -INFINITY;
+  }
+  float mc[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float m = x[32 * c];
+#pragma unroll
+    for (int k = 1; k < 31; k += 2) m = max3f(m, x[32 * c + k], x[32 * c + k + 1]);
+    mc[c] = fmaxf(m, x[32 * c + 31]);
+  }
+  const float mx = max3f(mc[0], mc[1], fmaxf(mc[2], mc[3]));
+  const float m_tile = INT8 ? (mx - 12582912.0f) * sc : mx * sc;
+  const float m_new = fmaxf(m_run, m_tile);
+  const bool need = m_new > m_run + 8.0f;
+  const bool rescale = __any_sync(0xffffffffu, need);
+  float alpha = 1.f;
+  if (need) {
+    alpha = ex2_approx(m_run - m_new);
+    l_run *= alpha;
+    m_run = m_new;
+  }
+  const float m_use = m_run == -INFINITY ? 0.f : m_run;
+  const float2 sc2 = make_float2(sc, sc), cst2 = make_float2(-m_use, -m_use);
+  const float2 off2 = make_float2(-12582912.0f, -12582912.0f);
+  float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
+  uint32_t pk[64];
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const int col = 2 * i;
+    float2 xv = make_float2(x[col], x[col + 1]);
+    if constexpr (INT8) xv = fadd2(xv, off2);
+    const float2 a = ffma2(xv, sc2, cst2);
+    const float p0 = ex2_approx(a.x), p1 = ex2_approx(a.y);
+    if (i & 1)
+      ls1 = fadd2(ls1, make_float2(p0, p1));
+    else
+      ls0 = fadd2(ls0, make_float2(p0, p1));
+    pk[i] = pack2(p0, p1, FP16);
+  }
+  l_run += (ls0.x + ls0.y) + (ls1.x + ls1.y);
+  if (j > 0) {
+    bool ok = mbar_wait(pv_done_t, (j - 1) & 1, abort_flag, W_SOFTMAX + 5);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+  }
+  // 16-byte chunk c (8 keys) of the row goes to chunk c ^ (row % 8) of its panel row
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint32_t a = p_row + (uint32_t)(c >> 3) * (128 * 128) + ((((uint32_t)c & 7u) ^ p_xor) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
+                 "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3]));
+  }
+  if (rescale && j > 0) {
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + 32 * c, o);
+      tmem_ld_wait(o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+      tmem_st32(tO + 32 * c, o);
+    }
+  }
+  return true;
+}
+
 template <int D, int QK, bool FP16, bool SPLIT>
 __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -477,7 +603,9 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* drain = o_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* s_free = drain + 1;    // P in shared memory only
+  uint64_t* pv_done = s_free + 2;  // P in shared memory only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -488,6 +616,8 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], TATTN_PFULL_PER_WARP ? R::kThreadsPerTile / 32 : R::kThreadsPerTile);
       mbar_init(&o_done[i], 1);
+      mbar_init(&s_free[i], R::kThreadsPerTile / 32);
+      mbar_init(&pv_done[i], 1);
     }
     for (int i = 0; i < C::KSTAGES; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < C::VSTAGES; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
@@ -612,6 +742,73 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
           mbar_wait(&k_full[j % C::KSTAGES], (j / C::KSTAGES) & 1, nullptr, W_DRAIN + 2, 200000000ull);
         for (int j = max(0, v_issued - C::VSTAGES); j < v_issued; ++j)
           mbar_wait(&v_full[j % C::VSTAGES], (j / C::VSTAGES) & 1, nullptr, W_DRAIN + 3, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == R::kMmaWarp && C::PSMEM) {
+    // ======================= MMA issuer, P in shared memory (event-driven) =======================
+    // Four in-order streams: per query tile t, S_t(j) = Q_t K(j)^T (needs K(j) and S_t read out by
+    // the softmax: s_free) and O_t += P_t(j) V(j) (needs P_t(j): p_full, and V(j)).  One thread
+    // polls them with non-blocking tests and issues whatever is ready, so no stream waits behind
+    // another.  A K or V stage is released after its last consumer (the later of the two tiles).
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      const uint32_t p_addr = smem_u32(smem + C::OFF_P);
+      int qj0 = 0, qj1 = 0, pj0 = 0, pj1 = 0;  // next Q K^T / P V index of each tile
+      bool ok = true;
+      unsigned long long t_idle = 0;
+      uint32_t spins = 0;
+      while (pj0 < n0 || pj1 < n1) {
+        bool did = false;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int nt = t ? n1 : n0, no = t ? n0 : n1;
+          int& qj = t ? qj1 : qj0;
+          int& pj = t ? pj1 : pj0;
+          const int qo = t ? qj0 : qj1, po = t ? pj0 : pj1;
+          if (pj < qj) {  // O_t += P_t(pj) V(pj)
+            const int j = pj, vs = j % C::VSTAGES;
+            if (mbar_test(&p_full[t], j & 1) && mbar_test(&v_full[vs], (j / C::VSTAGES) & 1)) {
+              tc_fence_after();
+              issue_pv_ss<D, FP16>(tmem + C::tm_o(t), p_addr + t * C::P_TILE, v_addr + vs * C::V_TILE, j > 0);
+              mma_commit(&pv_done[t]);
+              if (j + 1 == nt) mma_commit(&o_done[t]);  // the tile's last P V: O is final
+              if (j >= no || po > j) mma_commit(&v_empty[vs]);  // the other tile is done with V(j)
+              ++pj;
+              did = true;
+            }
+          }
+          if (qj < nt) {  // S_t(qj) = Q_t K(qj)^T
+            const int j = qj, ks = j % C::KSTAGES;
+            if ((j == 0 ? mbar_test(&q_full[t], 0) : mbar_test(&s_free[t], (j - 1) & 1)) &&
+                mbar_test(&k_full[ks], (j / C::KSTAGES) & 1)) {
+              tc_fence_after();
+              issue_qk<D, QK, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr + ks * C::K_TILE);
+              mma_commit(&s_full[t]);
+              if (j >= no || qo > j) mma_commit(&k_empty[ks]);  // the other tile is done with K(j)
+              ++qj;
+              did = true;
+            }
+          }
+        }
+        // bounded: no progress for kWaitTimeoutNs (or another role's abort) ends the loop
+        if (did) {
+          spins = 0;
+        } else if ((++spins & 63u) == 0u) {
+          if (*abort_flag) { ok = false; break; }
+          const unsigned long long now = globaltimer_ns();
+          if (spins == 64u) t_idle = now;
+          else if (now - t_idle > kWaitTimeoutNs) {
+            report_timeout(abort_flag, W_MMA + 7);
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (!ok) {
+        // Drain: wait until every MMA issued so far has completed before TMEM is released.
+        mma_commit(drain);
+        mbar_wait(drain, 0, nullptr, W_DRAIN + 4, 200000000ull);
       }
     }
     __syncwarp();
@@ -777,6 +974,9 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       // row prefix mask: this row's limit, and the tile-wide smallest limit (rows < N)
       const int row_lim = (p.row_lim != nullptr && row < p.N) ? min(max(__ldg(&p.row_lim[row]), 0), p.Nk) : 0;
       const int tile_min_lim = p.row_lim != nullptr ? lim_stats[2 * t + 1] : INT_MAX;
+      // (P in shared memory) this thread's row of the tile's P buffer, and its swizzle key
+      const uint32_t p_row = smem_u32(smem + C::OFF_P) + (uint32_t)(t * C::P_TILE) + (uint32_t)(wq * 32 + lane) * 128u;
+      const uint32_t p_xor = (uint32_t)(lane & 7);
       bool ok = true;
       for (int j = 0; j < nt; ++j) {
         ok = mbar_wait(&s_full[t], j & 1, abort_flag, W_SOFTMAX + 1);
@@ -790,13 +990,26 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         // [0, lim) of the tile are visible
         const int col0 = j * 128;
         const bool diag = p.causal && (j == nt - 1);
-        if (diag || (col0 + 128 > p.Nk) || (col0 + 128 > tile_min_lim)) {
-          const int lim = (p.row_lim != nullptr ? row_lim : (diag ? min(row + 1, p.Nk) : p.Nk)) - col0;
-          ok = softmax_step<D, QK, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
+        if constexpr (C::PSMEM) {
+          if (diag || (col0 + 128 > p.Nk) || (col0 + 128 > tile_min_lim)) {
+            const int lim = (p.row_lim != nullptr ? row_lim : (diag ? min(row + 1, p.Nk) : p.Nk)) - col0;
+            ok = softmax_step_ps<D, QK, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &s_free[t], &pv_done[t], p_row,
+                                                    p_xor, abort_flag);
+          } else {
+            ok = softmax_step_ps<D, QK, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &s_free[t], &pv_done[t],
+                                                     p_row, p_xor, abort_flag);
+          }
+          if (!ok) break;
+          fence_async_smem();  // P (generic stores) before the MMA's async-proxy reads
         } else {
-          ok = softmax_step<D, QK, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
+          if (diag || (col0 + 128 > p.Nk) || (col0 + 128 > tile_min_lim)) {
+            const int lim = (p.row_lim != nullptr ? row_lim : (diag ? min(row + 1, p.Nk) : p.Nk)) - col0;
+            ok = softmax_step<D, QK, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
+          } else {
+            ok = softmax_step<D, QK, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
+          }
+          if (!ok) break;
         }
-        if (!ok) break;
         tmem_st_wait();
         tc_fence_before();
         if (TATTN_PFULL_PER_WARP) {

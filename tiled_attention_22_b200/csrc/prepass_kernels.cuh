@@ -126,7 +126,12 @@ __global__ void __launch_bounds__(4 * D, 256 / D) quant_kernel(const uint16_t* _
   const int T = (N + 127) / 128;
   const int nK = B * Hkv * T;
   const bool is_k = (int)blockIdx.x < nK;
-  const int blk = is_k ? blockIdx.x : blockIdx.x - nK;
+  // K blocks run last-to-first: the mean pass just streamed K first-to-last, so the end of K is
+  // what is still in L2 (K is often about the size of L2) and is read again first.
+#ifndef TATTN_QUANT_K_REVERSE
+#define TATTN_QUANT_K_REVERSE 1
+#endif
+  const int blk = is_k ? (TATTN_QUANT_K_REVERSE ? nK - 1 - (int)blockIdx.x : (int)blockIdx.x) : (int)blockIdx.x - nK;
   const int t = blk % T;
   const int bh = blk / T;  // b*Hkv + g for K, b*Hq + h for Q
   const int g_mean = is_k ? bh : (bh / Hq) * Hkv + (bh % Hq) / (Hq / Hkv);
