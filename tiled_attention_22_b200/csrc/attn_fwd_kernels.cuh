@@ -978,12 +978,27 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       const uint32_t p_row = smem_u32(smem + C::OFF_P) + (uint32_t)(t * C::P_TILE) + (uint32_t)(wq * 32 + lane) * 128u;
       const uint32_t p_xor = (uint32_t)(lane & 7);
       bool ok = true;
+      // 8-bit modes: the key block's scale, loaded one tile ahead so that its latency is off the
+      // tile's critical path
+#ifndef TATTN_SK_PREFETCH
+#define TATTN_SK_PREFETCH 1
+#endif
+      const float* skp = p.sk + (size_t)kvz * nkv;
+      float sk_next = (QUANT && TATTN_SK_PREFETCH && nt > 0) ? __ldg(skp) : 0.f;
       for (int j = 0; j < nt; ++j) {
+        float sk_j = 0.f;
+        if constexpr (QUANT) {
+          if (TATTN_SK_PREFETCH) {
+            sk_j = sk_next;
+            if (j + 1 < nt) sk_next = __ldg(skp + j + 1);
+          }
+        }
         ok = mbar_wait(&s_full[t], j & 1, abort_flag, W_SOFTMAX + 1);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        float sc = QUANT ? sq_scale * __ldg(&p.sk[(size_t)kvz * nkv + j]) : sq_scale;
+        if (QUANT && !TATTN_SK_PREFETCH) sk_j = __ldg(skp + j);
+        float sc = QUANT ? sq_scale * sk_j : sq_scale;
         if constexpr (QUANT) sc = fmaxf(sc, 1e-30f);  // a zero block: keep -inf * sc = -inf for masks
         // causal diagonal tile (key > query), the ragged last key tile (key >= Nk) and, under a
         // row prefix mask, every tile that reaches past some row's limit are masked; keys
