@@ -388,7 +388,9 @@ def run_native(args, w, world, rank, local):
             "int8_qk": {"tflops": r8["tflops"], "ms_per_step": r8["ms_per_step"],
                         "prepass_ms": r8["kernel_ms"][0], "fused_ms": fused_ms,
                         "fused_tflops": achieved,
-                        "prepass_gbs": _prepass_bytes(w) / (r8["kernel_ms"][0] * 1e-3) / 1e9},
+                        "prepass_gbs": _prepass_bytes(w) / (r8["kernel_ms"][0] * 1e-3) / 1e9,
+                        "prepass_frac_of_hbm_peak": _prepass_bytes(w) / (r8["kernel_ms"][0] * 1e-3) / 1e9
+                        / peaks["hbm_gbs"]},
             "fp8_qk": {"tflops": rf["tflops"], "ms_per_step": rf["ms_per_step"],
                        "prepass_ms": rf["kernel_ms"][0], "fused_ms": rf["kernel_ms"][1],
                        "fused_tflops": flops / (rf["kernel_ms"][1] * 1e-3) / 1e12,
@@ -515,11 +517,11 @@ def _fused_bytes(w, mode):
 
 
 def _prepass_bytes(w):
-    """Algorithmic bytes of the pre-pass: K read twice (mean, quantise) and written as int8; Q read once,
-    written as int8; scales, mean and lse bias are small."""
+    """Algorithmic bytes of the pre-pass: K and Q each read once in 16-bit and written once as 8-bit
+    codes, plus the lse bias (4 B per query row); scales and the mean are small."""
     nk = w.B * w.Hkv * w.N * w.d
     nq = w.B * w.Hq * w.N * w.d
-    return 2 * nk * 2 + nk + 2 * nq + nq + 4 * w.B * w.Hq * w.N
+    return 3 * nk + 3 * nq + 4 * w.B * w.Hq * w.N
 
 
 def main():

@@ -75,6 +75,8 @@ PREPASS = [
     (1, 3, 1, 1, 64, "bf16", "normal"),
     (1, 2, 2, 515, 64, "fp16", "outlier_channels"),
     (1, 4, 2, 2048, 128, "bf16", "k_offset"),
+    (1, 8, 1, 16384, 128, "bf16", "k_offset"),  # 8 query heads on one kv head
+    (1, 2, 2, 16385, 64, "fp16", "normal"),     # one-token ragged tail
 ]
 
 

@@ -140,6 +140,10 @@ PREPASS = [
     (1, 3, 1, 1, 64, "bf16", "normal"),
     (1, 2, 2, 515, 64, "fp16", "outlier_channels"),
     (1, 4, 2, 2048, 128, "bf16", "k_offset"),
+    # many short units; 16 query heads on one kv head (16K tokens); a one-token ragged tail
+    (8, 8, 8, 256, 128, "bf16", "normal"),
+    (1, 16, 1, 16384, 128, "bf16", "k_offset"),
+    (1, 2, 2, 16385, 64, "fp16", "normal"),
 ]
 
 
