@@ -414,6 +414,7 @@ def run_native(args, w, world, rank, local):
     if not args.no_decode:
         line["decode"] = run_decode(args, dev, world, peaks)
         line["prefix_mask"] = run_prefix_mask(args, dev, world, peaks)
+        line["context_parallel"] = run_context_parallel(args, dev, world, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     return line
@@ -505,6 +506,60 @@ def run_prefix_mask(args, dev, world, peaks):
     return out
 
 
+def run_context_parallel(args, dev, world, peaks, ranks=4):
+    """Context-parallel (ring) attention on the 131K-token GQA workload split over ``ranks`` ranks,
+    emulated on this GPU: each rank's steps (fused kernel + lse merge per visible key block) run
+    back to back with the blocks already split; no exchange (its NVLink cost is not measured).
+    Reported beside one fused-kernel call over the whole sequence, both in bf16_exact."""
+    import tiled_attention_22_b200 as ta
+    from tiled_attention_22_b200.ring import ring_rank_emulated, ring_schedule
+
+    w = WORKLOADS[5]
+    q, k, v = (t.to(dev) for t in make_inputs(w))
+    n = w.N // ranks
+    qs = [q[:, :, r * n:(r + 1) * n].contiguous() for r in range(ranks)]
+    kv = [(k[:, :, j * n:(j + 1) * n].contiguous(), v[:, :, j * n:(j + 1) * n].contiguous()) for j in range(ranks)]
+    flops = w.flops()
+
+    def ring():
+        for r in range(ranks):
+            ring_rank_emulated(qs[r], kv, r, causal=w.causal, scale=w.scale)
+
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), device=dev, dtype=torch.float32)
+
+    def whole():
+        ta.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+
+    res = {}
+    for name, fn in (("ring", ring), ("single_call", whole)):
+        fn()
+        torch.cuda.synchronize()
+        _barrier(world)
+        n_calls = 3
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_calls):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        _barrier(world)
+        res[name] = _max_over_ranks(e0.elapsed_time(e1), world, dev) / n_calls
+    if ta.attn_check_status() != 0:
+        raise RuntimeError("device-side wait timed out in the context-parallel benchmark")
+    steps = sum(kind != "skip" for r in range(ranks) for _, _, kind in ring_schedule(r, ranks, w.causal))
+    tf = flops / (res["ring"] * 1e-3) / 1e12
+    out = {w.name + f"_ring{ranks}": {
+        "ms_per_call": res["ring"], "TFLOP/s": tf * world, "frac_of_bf16_peak": tf / peaks["bf16_sustained"],
+        "single_call_ms": res["single_call"], "ring_over_single": res["ring"] / res["single_call"],
+        "launches_per_call": 2 * steps, "kernels": "attn_fwd_kernel<128,bf16> + lse_merge_kernel<128,bf16>",
+        "note": "all ranks' steps on one GPU; the key/value exchange over NVLink is not timed"}}
+    out["peak_note"] = "bf16 dense GEMM %.0f TFLOP/s (%s, sustained)" % (peaks["bf16_sustained"], peaks["source"])
+    del q, k, v, qs, kv, o
+    torch.cuda.empty_cache()
+    return out
+
+
 def _fused_bytes(w, mode):
     """Algorithmic bytes of one fused-kernel launch: Q and K read once (1 B/elt as INT8 codes,
     2 B/elt in bf16_exact), V read once, O written once, lse written (4 B/row); scales and the
@@ -533,7 +588,7 @@ def main():
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true", help="skip the KV-cache decode measurements")
+    ap.add_argument("--no-decode", action="store_true", help="skip the measurements of the other paths (KV-cache decode, prefix mask, ring)")
     ap.add_argument("--modes", default="int8_qk,bf16_exact,fp8_qk",
                     help="modes to time (the headline value is int8_qk; drop one only for profiling)")
     args = ap.parse_args()

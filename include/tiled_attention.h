@@ -268,6 +268,30 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
 int attn_check_status(void);
 
 /*
+ * attn_merge_lse - joins two attention results over disjoint key sets by their log-sum-exp, the
+ * step a sequence-parallel (ring) attention takes after each exchange.  The "FlashAttention"
+ * glossary (deep-dive section, FAQ) rescales partial softmax results by running maxima and sums;
+ * for results (O_a, lse_a) and (O_b, lse_b) over key sets A and B the result over A u B is
+ *     lse = ln(exp(lse_a) + exp(lse_b)),  O = exp(lse_a - lse) O_a + exp(lse_b - lse) O_b,
+ * which is what ring attention (named by the APB article as the exact sequence-parallel
+ * baseline) computes after each step.  Float32 arithmetic, one pass over HBM.
+ *
+ *   rows    number of query rows (B * Hq * Nq); each row holds d values (d = 64 or 128).
+ *   o_acc   [rows, d] float32, lse_acc [rows] float32: the running result (device, read and
+ *           written).  A row whose lse is -inf has no keys: its O must be 0; it adds no weight.
+ *   o_part  [rows, d] 16-bit (dtype), lse_part [rows] float32: one step's result, e.g. the o and
+ *           lse outputs of attn_fwd for the same rows (natural-log lse).  Both NULL: nothing is
+ *           merged (use with o_out to convert the running result).
+ *   first   1: o_acc / lse_acc are set to the part (their contents are ignored); 0: merged.
+ *   o_out   [rows, d] 16-bit (dtype) or NULL: receives the merged O rounded to nearest even.
+ *   All pointers device, 16-byte aligned; rows = 0 launches nothing.  Errors: ATTN_ERR_ARG
+ *   (null accumulator, first without a part, only one of o_part / lse_part, bad dtype or
+ *   first), ATTN_ERR_UNSUPPORTED (d), ATTN_ERR_ALIGN.
+ */
+int attn_merge_lse(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                   void* o_out, long long rows, int d, int dtype, int first, void* stream);
+
+/*
  * attn_test_wait_timeout - test hook for failure detection.  Launches one tiny kernel whose single
  * thread waits on an mbarrier that nothing ever completes, with a limit of `limit_us`
  * microseconds (1..1000000).  The wait gives up, sets the device status word and the kernel

@@ -1,0 +1,84 @@
+"""Context-parallel (ring) attention, host side on CPU: the schedule, and the key/value exchange
+over gloo ranks (2 and 3 processes) with the same ring_pass_blocks code the GPU path runs over
+NCCL.  The attention arithmetic of each step is checked on the GPU (test_gpu_ring.py)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from tiled_attention_22_b200.ring import ring_pass_blocks, ring_schedule
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("causal", [False, True])
+def test_schedule_visits_every_block_once(world, causal):
+    for r in range(world):
+        sched = ring_schedule(r, world, causal)
+        assert [s for s, _, _ in sched] == list(range(world))
+        assert sorted(j for _, j, _ in sched) == list(range(world))
+        for s, j, kind in sched:
+            assert j == (r - s) % world
+            if not causal:
+                assert kind == "full"
+            else:
+                # the diagonal block at step 0, earlier blocks unmasked, later blocks invisible
+                assert kind == ("causal" if j == r else "full" if j < r else "skip")
+        if causal:
+            # rank r sees blocks 0..r: r + 1 useful steps, the last at step r
+            useful = [s for s, _, kind in sched if kind != "skip"]
+            assert useful == list(range(r + 1))
+
+
+def test_schedule_rejects_bad_rank():
+    with pytest.raises(ValueError):
+        ring_schedule(3, 3, True)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _block(rank, shape):
+    k = torch.arange(torch.Size(shape).numel(), dtype=torch.float32).reshape(shape) + 1000.0 * rank
+    return k, -k
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        shape = (2, 3, 5, 4)
+        k, v = _block(rank, shape)
+        k0, v0 = k.clone(), v.clone()
+        seen = []
+
+        def on_step(s, j, kj, vj):
+            seen.append((s, j, kj.clone(), vj.clone()))
+
+        ring_pass_blocks(k, v, on_step)
+        res = []
+        for s, j, kj, vj in seen:
+            ek, ev = _block(j, shape)
+            res.append((s, j, bool(torch.equal(kj, ek)), bool(torch.equal(vj, ev))))
+        out[rank] = (res, bool(torch.equal(k, k0) and torch.equal(v, v0)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_ring_delivers_block_r_minus_s(world):
+    out = mp.Manager().dict()
+    mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
+    for r in range(world):
+        res, untouched = out[r]
+        assert untouched, f"rank {r}: its own block was overwritten"
+        assert [s for s, _, _, _ in res] == list(range(world))
+        for s, j, k_ok, v_ok in res:
+            assert j == (r - s) % world
+            assert k_ok and v_ok, f"rank {r} step {s}: block {j} arrived wrong"

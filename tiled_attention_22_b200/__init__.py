@@ -1,5 +1,6 @@
 """B200 (sm_100a) tiled attention forward: bf16_exact, SageAttention-style int8_qk and fp8_qk,
-a row-prefix-masked variant (the APB mask shape) and a KV-cache decode path.
+a row-prefix-masked variant (the APB mask shape), a KV-cache decode path, and context-parallel
+(ring) attention over torch.distributed with log-sum-exp merges (``ring``).
 
 The computation runs in the CUDA library built from ``csrc/`` (C ABI in
 ``include/tiled_attention.h``); this package only marshals arguments.
@@ -24,6 +25,7 @@ from .binding import (  # noqa: F401
     attn_fwd_fp8_quantized,
     attn_fwd_int8_quantized,
     attn_fwd_prefix_masked,
+    attn_merge_lse,
     attn_probe_qk_int32,
     attn_quant_scratch_bytes,
     attn_quant_smooth_k,

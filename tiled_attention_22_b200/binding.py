@@ -44,6 +44,7 @@ _SIGNATURES = {
     "attn_fwd_prefix_masked": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _f, _i, _vp]),
     "attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _sz, _vp]),
     "attn_decode_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "attn_merge_lse": (_i, [_vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, _i, _i, _i, _vp]),
     "attn_check_status": (_i, []),
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_last_cuda_error": (ctypes.c_char_p, []),
@@ -355,6 +356,35 @@ def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, dq, dk, dv, do_, dls
                            MODES[mode], DTYPES[q_host.dtype], _ptr(workspace),
                            0 if workspace is None else workspace.numel(), _stream(stream))
     _check(rc, "attn_fwd_host")
+
+
+def attn_merge_lse(o_acc, lse_acc, o_part=None, lse_part=None, out=None, first=False, stream=None):
+    """Join a partial attention result (o_part 16-bit [..., d], lse_part float32 [...]) into the
+    running result (o_acc float32 [..., d], lse_acc float32 [...]) by their log-sum-exp, in place;
+    ``first`` sets the running result to the part; ``out`` (16-bit, like o_part) receives the
+    merged O.  Returns ``out``."""
+    lib = load_library()
+    if o_acc.dtype != torch.float32 or lse_acc.dtype != torch.float32:
+        raise ValueError("o_acc and lse_acc must be float32")
+    d = o_acc.shape[-1]
+    rows = o_acc.numel() // d
+    if lse_acc.numel() != rows:
+        raise ValueError("lse_acc must hold one value per row of o_acc")
+    ref = o_part if o_part is not None else out
+    if ref is None:
+        raise ValueError("nothing to do: give o_part/lse_part, out, or both")
+    for t in (o_acc, lse_acc, o_part, lse_part, out):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("every tensor must be a contiguous CUDA tensor")
+    for t in (o_part, out):
+        if t is not None and (t.dtype not in DTYPES or t.dtype != ref.dtype or t.numel() != rows * d):
+            raise ValueError("o_part and out must be 16-bit tensors of o_acc's size and one dtype")
+    if lse_part is not None and (lse_part.dtype != torch.float32 or lse_part.numel() != rows):
+        raise ValueError("lse_part must be float32 with one value per row")
+    rc = lib.attn_merge_lse(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part), _ptr(out), rows, d,
+                            DTYPES[ref.dtype], int(bool(first)), _stream(stream))
+    _check(rc, "attn_merge_lse")
+    return out
 
 
 def attn_check_status() -> int:

@@ -17,6 +17,7 @@
 
 #include "attn_fwd_kernels.cuh"
 #include "decode_kernels.cuh"
+#include "merge_kernels.cuh"
 #include "prepass_kernels.cuh"
 
 namespace {
@@ -502,6 +503,34 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   p.part_lse = reinterpret_cast<float*>(ws + w.part_lse);
   p.unit_arrived = reinterpret_cast<unsigned int*>(ws + w.unit_arrived);
   return launch_decode(q, k_cache, v_cache, dtype, ctas, p, static_cast<cudaStream_t>(stream));
+}
+
+int attn_merge_lse(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out,
+                   long long rows, int d, int dtype, int first, void* stream) {
+  if (!o_acc || !lse_acc || rows < 0 || (first != 0 && first != 1)) return ATTN_ERR_ARG;
+  if (first && (!o_part || !lse_part)) return ATTN_ERR_ARG;
+  if ((o_part == nullptr) != (lse_part == nullptr)) return ATTN_ERR_ARG;
+  if (dtype != ATTN_BF16 && dtype != ATTN_FP16) return ATTN_ERR_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(o_acc) || !aligned16(lse_acc) || (o_part && !aligned16(o_part)) ||
+      (lse_part && !aligned16(lse_part)) || (o_out && !aligned16(o_out)))
+    return ATTN_ERR_ALIGN;
+  if (rows == 0) return ATTN_OK;
+  const long long want = (rows + 7) / 8;  // 8 rows (one per warp) per CTA of 256 threads
+  const unsigned grid = (unsigned)std::min<long long>(want, (long long)device_sm_count() * 16);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto* part = static_cast<const uint16_t*>(o_part);
+  auto* out = static_cast<uint16_t*>(o_out);
+  const bool fp16 = dtype == ATTN_FP16;
+  if (d == 128) {
+    if (fp16) lse_merge_kernel<128, true><<<grid, 256, 0, st>>>(o_acc, lse_acc, part, lse_part, out, rows, first);
+    else lse_merge_kernel<128, false><<<grid, 256, 0, st>>>(o_acc, lse_acc, part, lse_part, out, rows, first);
+  } else {
+    if (fp16) lse_merge_kernel<64, true><<<grid, 256, 0, st>>>(o_acc, lse_acc, part, lse_part, out, rows, first);
+    else lse_merge_kernel<64, false><<<grid, 256, 0, st>>>(o_acc, lse_acc, part, lse_part, out, rows, first);
+  }
+  TATTN_CUDA(cudaGetLastError());
+  return ATTN_OK;
 }
 
 int attn_check_status(void) {
