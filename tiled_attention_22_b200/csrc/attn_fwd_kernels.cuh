@@ -117,11 +117,16 @@ struct FwdCfg {
                                        : (D == 128 ? (BYTE ? TATTN_VS_128I : TATTN_VS_128B) : 4);
   static constexpr int P_PANEL_BYTES = 128 * 128;              // 128 rows x 64 keys x 2 B
   static constexpr int P_TILE = PSMEM ? 2 * P_PANEL_BYTES : 0;
+  // O staging for the epilogue's TMA stores: one 32-row x 64-column 16-bit slot (4 KB, 128-byte
+  // swizzle) per softmax warp; a warp stores its 32 rows panel by panel through its slot
+  static constexpr int O_SLOT = 32 * 128;
+  static constexpr int O_STAGE = PSMEM ? 0 : 8 * O_SLOT;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_P = OFF_Q + QT * Q_TILE;
   static constexpr int OFF_K = OFF_P + QT * P_TILE;
   static constexpr int OFF_V = OFF_K + KSTAGES * K_TILE;
-  static constexpr int OFF_BAR = OFF_V + VSTAGES * V_TILE;
+  static constexpr int OFF_O = OFF_V + VSTAGES * V_TILE;
+  static constexpr int OFF_BAR = OFF_O + O_STAGE;
   // barriers: q_full[2] k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2] o_done[2]
   // drain, then (P in shared memory) s_free[2] pv_done[2]
   static constexpr int NBAR = 2 + 2 * KSTAGES + 2 * VSTAGES + 6 + 1 + 4;
@@ -587,7 +592,8 @@ __device__ __forceinline__ bool softmax_step_ps(uint32_t tS, uint32_t tO, float 
 template <int D, int QK, bool FP16, bool SPLIT>
 __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const FwdParams p) {
   constexpr bool QUANT = QK != QK_F16;  // 8-bit codes with per-block scales sq, sk and the lse bias
   using C = FwdCfg<D, QUANT>;
   using R = FwdRoles<SPLIT>;
@@ -633,6 +639,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
   }
   tc_fence_before();
   __syncthreads();
@@ -985,6 +992,8 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
 #endif
       const float* skp = p.sk + (size_t)kvz * nkv;
       float sk_next = (QUANT && TATTN_SK_PREFETCH && nt > 0) ? __ldg(skp) : 0.f;
+      // 8-bit modes: the row's lse bias, loaded now so that the epilogue does not wait for it
+      const float lse_bias = (QUANT && p.lse != nullptr && nt > 0 && row < p.N) ? __ldg(&p.bias[(size_t)bh * p.N + row]) : 0.f;
       for (int j = 0; j < nt; ++j) {
         float sk_j = 0.f;
         if constexpr (QUANT) {
@@ -1050,25 +1059,63 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
           tc_fence_after();
           // (a row that saw no key, possible only under a row prefix mask, has l = 0: O = 0)
           const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-          uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)bh * p.N + (size_t)row) * (D * 2);
-  #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * c, o);
-            tmem_ld_wait(o);
-            uint32_t pk[16];
-  #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, FP16);
-            if (row < p.N) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
-  #pragma unroll
-              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          if constexpr (C::O_STAGE > 0) {
+            // O through this warp's shared-memory slot, one 64-column panel at a time, each
+            // panel written to global memory by one TMA store of the warp's 32 rows (rows past
+            // N are clipped by the tensor map).  Slot layout: row r at r * 128 bytes, 16-byte
+            // chunk c at position c ^ (r & 7) (the 128-byte swizzle of the tensor map).
+            uint8_t* slot = smem + C::OFF_O + warp * C::O_SLOT;
+            const uint32_t swz = (uint32_t)(lane & 7);
+            const int y0 = row0 + wq * 32;
+#pragma unroll
+            for (int pn = 0; pn < D / 64; ++pn) {
+              if (pn > 0) {  // the previous panel's store has finished reading the slot
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+              }
+#pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                uint32_t o[32];
+                tmem_ld32(tO + 64 * pn + 32 * cc, o);
+                tmem_ld_wait(o);
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  pk[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, FP16);
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                  *reinterpret_cast<uint4*>(slot + lane * 128 + (((uint32_t)(cc * 4 + v) ^ swz) << 4)) =
+                      make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              }
+              fence_async_smem();  // the slot's generic stores before the TMA engine reads it
+              __syncwarp();
+              if (lane == 0 && y0 < p.N) {
+                tma_store_3d(&tmO, slot, pn * 64, y0, bh);
+                bulk_commit_group();
+              }
+            }
+          } else {
+            uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + ((size_t)bh * p.N + (size_t)row) * (D * 2);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tO + 32 * c, o);
+              tmem_ld_wait(o);
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l, FP16);
+              if (row < p.N) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                  dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              }
             }
           }
           if (p.lse != nullptr && row < p.N) {
             float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-            if constexpr (QUANT) lse += p.bias[(size_t)bh * p.N + row];
+            if constexpr (QUANT) lse += lse_bias;
             p.lse[(size_t)bh * p.N + row] = lse;
           }
         }
@@ -1076,6 +1123,11 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       if (!ok) {
         // make sure this thread's TMEM traffic is finished before teardown
         tmem_st_wait();
+      }
+      if constexpr (C::O_STAGE > 0) {
+        // the slot must stay until the last store has read it
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
       }
     }
   }

@@ -12,7 +12,7 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
   using C = FwdCfg<D, BYTE>;
   constexpr bool SPLIT = TATTN_SPLIT != 0;
   using R = FwdRoles<SPLIT>;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const CUtensorMapDataType qk_dt =
       BYTE ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : (FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
   const CUtensorMapDataType v_dt = FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -20,6 +20,8 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
   if ((rc = make_map(&tq, q, qk_dt, C::QK_ELEM, D, p.N, p.B * p.Hq, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
   if ((rc = make_map(&tk, k, qk_dt, C::QK_ELEM, D, p.Nk, p.B * p.Hkv, C::QK_BOX_X, swizzle_for(C::QK_ROW)))) return rc;
   if ((rc = make_map(&tv, v, v_dt, 2, D, p.Nk, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+  // O: the epilogue's stores, 64 columns x 32 rows (one softmax warp's rows) per box
+  if ((rc = make_map(&to, p.o, v_dt, 2, D, p.N, p.B * p.Hq, 64, CU_TENSOR_MAP_SWIZZLE_128B, 32))) return rc;
   auto kern = attn_fwd_kernel<D, QK, FP16, SPLIT>;
   // Once per device: allow the dynamic shared memory, and check the register split.  The kernel
   // moves registers between warpgroups with setmaxnreg; the increase only completes if the
@@ -42,7 +44,7 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
     checked[dev].store(1, std::memory_order_release);
   }
   const long long grid = (long long)p.n_mblocks * p.B * p.Hq;
-  kern<<<(unsigned)grid, R::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  kern<<<(unsigned)grid, R::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   TATTN_CUDA(cudaGetLastError());
   return ATTN_OK;
 }
