@@ -339,3 +339,31 @@ def test_kernel_exp2_against_cuda_exp2f(ta, use_poly):
     assert torch.isfinite(y).all()
     if use_poly:
         assert torch.equal(ta.attn_test_exp2(x, 2), y)  # packed pairs: the same bits
+
+
+def test_persistent_path_deterministic_and_stream_safe(ta):
+    """16-bit Q K^T at d = 128 runs on persistent CTAs that take work items from a per-stream ticket
+    counter: the bytes must not depend on which CTA took which item (two calls agree), and calls on
+    two streams at once (two counters) must give the bytes of the same calls made one by one."""
+    w1 = Workload("p1", 2, 8, 2, 1000, 128, True, "bf16", "normal", 95000)
+    w2 = Workload("p2", 1, 16, 16, 777, 128, False, "bf16", "k_offset", 95010)
+    ins = [[t.cuda() for t in make_inputs(w)] for w in (w1, w2)]
+    ref = []
+    for (q, k, v), w in zip(ins, (w1, w2)):
+        ref.append(ta.attn_fwd(q, k, v, causal=w.causal))
+    again = ta.attn_fwd(*ins[0], causal=w1.causal)
+    torch.cuda.synchronize()
+    assert torch.equal(again[0], ref[0][0]) and torch.equal(again[1], ref[0][1])
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for s, (q, k, v), w in zip(streams, ins, (w1, w2)):
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            outs.append([ta.attn_fwd(q, k, v, causal=w.causal, stream=s) for _ in range(3)])
+    torch.cuda.synchronize()
+    assert ta.attn_check_status() == 0
+    for got, (o, l) in zip(outs, ref):
+        for go, gl in got:
+            assert torch.equal(go, o) and torch.equal(gl, l)
+    O, L = oracle.attention(ins[0][0].cpu(), ins[0][1].cpu(), ins[0][2].cpu(), w1.scale, True)
+    assert_bf16(_np(ref[0][0]), ref[0][1].cpu().numpy().astype(np.float64), O, L, "persistent")

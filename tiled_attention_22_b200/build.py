@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 LIB_DIR = os.path.join(HERE, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libtiled_attention.so")
 SOURCES = ["csrc/api.cu"]
-DEPS = ["csrc/api.cu", "csrc/attn_fwd_kernels.cuh", "csrc/attn_fwd_launch.cuh", "csrc/tma_host.cuh",
+DEPS = ["csrc/api.cu", "csrc/attn_fwd_kernels.cuh", "csrc/attn_fwd_persistent.cuh", "csrc/attn_fwd_launch.cuh", "csrc/tma_host.cuh",
         "csrc/decode_kernels.cuh", "csrc/decode_launch.cuh", "csrc/merge_kernels.cuh", "csrc/prepass_kernels.cuh", "csrc/ptx.cuh",
         "../include/tiled_attention.h"]
 

@@ -16,6 +16,7 @@
 #include "tiled_attention.h"
 
 #include "attn_fwd_kernels.cuh"
+#include "attn_fwd_persistent.cuh"
 #include "decode_kernels.cuh"
 #include "merge_kernels.cuh"
 #include "prepass_kernels.cuh"
@@ -52,8 +53,8 @@ int check_shape(int B, int Hq, int Hkv, int N, int d) {
 }
 
 #include "tma_host.cuh"
-#include "attn_fwd_launch.cuh"
 #include "decode_launch.cuh"
+#include "attn_fwd_launch.cuh"
 
 int check_common(const void* q, const void* k, const void* v, const void* o, const float* lse, int B, int Hq,
                  int Hkv, int N, int d, int causal, float scale, int dtype) {

@@ -1,10 +1,69 @@
 #pragma once
-// attn_fwd_launch.cuh - host-side launch of the fused attention kernel: TMA descriptors for Q, K, V,
-// one-time per-device kernel setup (shared memory size, register-split check) and the grid.
-// Included by api.cu inside its anonymous namespace (after cuda_fail / TATTN_CUDA).
+// attn_fwd_launch.cuh - host-side launch of the fused attention kernel: TMA descriptors for Q, K, V
+// and O, one-time per-device kernel setup (shared memory size, register-split check), the choice
+// between one CTA per work item and persistent CTAs, and the grid.  Included by api.cu inside its
+// anonymous namespace (after cuda_fail / TATTN_CUDA and device_sm_count).
 #ifndef TATTN_SPLIT
 #define TATTN_SPLIT 0
 #endif
+
+// Persistent launches take their work items from a ticket counter, one per (device, stream) so that
+// launches on different streams never share one; it is cleared on the stream before each launch.
+// The counters live in the library, kTicketSlots per device; launches from further streams use one
+// CTA per item instead (the same results).
+constexpr int kTicketSlots = 256;
+__device__ unsigned g_fwd_tickets[kTicketSlots];
+
+unsigned* fwd_ticket_counter(cudaStream_t stream) {
+  static std::mutex mu;
+  static unsigned* base[kMaxDevices];
+  static cudaStream_t owner[kMaxDevices][kTicketSlots];
+  static int used[kMaxDevices];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (base[dev] == nullptr) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_fwd_tickets) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    base[dev] = static_cast<unsigned*>(addr);
+  }
+  for (int i = 0; i < used[dev]; ++i)
+    if (owner[dev][i] == stream) return base[dev] + i;
+  if (used[dev] == kTicketSlots) return nullptr;
+  owner[dev][used[dev]] = stream;
+  return base[dev] + used[dev]++;
+}
+
+// Once per device and kernel: allow the dynamic shared memory, and check the register split.  The
+// kernels move registers between warpgroups with setmaxnreg; the increase only completes if the
+// registers the CTA is launched with cover the split, so refuse to launch otherwise.
+template <class Kern>
+int setup_fwd_kernel(Kern kern, int smem_bytes, std::atomic<int>* checked) {
+  using R = FwdRoles<TATTN_SPLIT != 0>;
+  int dev = 0;
+  TATTN_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_LAUNCH;
+  if (checked[dev].load(std::memory_order_acquire) != 1) {
+    TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes));
+    cudaFuncAttributes attr;
+    TATTN_CUDA(cudaFuncGetAttributes(&attr, kern));
+    if ((long long)attr.numRegs * R::kThreads <
+            128LL * (R::kSoftmaxWarps / 4 * R::kRegsSoftmax + R::kRegsProducer) ||
+        attr.maxThreadsPerBlock < R::kThreads) {
+      std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                    "fused kernel built with %d registers/thread: too few for its register split", attr.numRegs);
+      return ATTN_ERR_LAUNCH;
+    }
+    checked[dev].store(1, std::memory_order_release);
+  }
+  return ATTN_OK;
+}
 
 template <int D, int QK, bool FP16>
 int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p, cudaStream_t stream) {
@@ -22,28 +81,29 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
   if ((rc = make_map(&tv, v, v_dt, 2, D, p.Nk, p.B * p.Hkv, 64, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
   // O: the epilogue's stores, 64 columns x 32 rows (one softmax warp's rows) per box
   if ((rc = make_map(&to, p.o, v_dt, 2, D, p.N, p.B * p.Hq, 64, CU_TENSOR_MAP_SWIZZLE_128B, 32))) return rc;
-  auto kern = attn_fwd_kernel<D, QK, FP16, SPLIT>;
-  // Once per device: allow the dynamic shared memory, and check the register split.  The kernel
-  // moves registers between warpgroups with setmaxnreg; the increase only completes if the
-  // registers the CTA is launched with cover the split, so refuse to launch otherwise.
-  static std::atomic<int> checked[kMaxDevices];
-  int dev = 0;
-  TATTN_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_LAUNCH;
-  if (checked[dev].load(std::memory_order_acquire) != 1) {
-    TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-    cudaFuncAttributes attr;
-    TATTN_CUDA(cudaFuncGetAttributes(&attr, kern));
-    if ((long long)attr.numRegs * R::kThreads <
-            128LL * (R::kSoftmaxWarps / 4 * R::kRegsSoftmax + R::kRegsProducer) ||
-        attr.maxThreadsPerBlock < R::kThreads) {
-      std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
-                    "fused kernel built with %d registers/thread: too few for its register split", attr.numRegs);
-      return ATTN_ERR_LAUNCH;
+  const long long items = (long long)p.n_mblocks * p.B * p.Hq;
+  // Persistent CTAs (one per SM) for 16-bit Q K^T at d = 128, where they measured 3-6% faster on
+  // the named workloads (the 8-bit modes and d = 64 measured no gain); not under a row prefix mask
+  // (its per-tile limits are read once per CTA) nor with the four-threads-per-row variant.
+  if constexpr (QK == QK_F16 && D == 128 && !SPLIT) {
+    unsigned* tickets = p.row_lim == nullptr && items <= 0x7fffffffll ? fwd_ticket_counter(stream) : nullptr;
+    if (tickets != nullptr) {
+      using PC = FwdPersistCfg<D, BYTE>;
+      auto pkern = attn_fwd_persistent_kernel<D, QK, FP16>;
+      static std::atomic<int> checked_p[kMaxDevices];
+      int rc2 = setup_fwd_kernel(pkern, PC::SMEM_BYTES, checked_p);
+      if (rc2) return rc2;
+      TATTN_CUDA(cudaMemsetAsync(tickets, 0, sizeof(unsigned), stream));
+      const long long grid = std::min<long long>(items, device_sm_count());
+      pkern<<<(unsigned)grid, R::kThreads, PC::SMEM_BYTES, stream>>>(tq, tk, tv, to, p, (int)items, tickets);
+      TATTN_CUDA(cudaGetLastError());
+      return ATTN_OK;
     }
-    checked[dev].store(1, std::memory_order_release);
   }
-  const long long grid = (long long)p.n_mblocks * p.B * p.Hq;
+  auto kern = attn_fwd_kernel<D, QK, FP16, SPLIT>;
+  static std::atomic<int> checked[kMaxDevices];
+  if ((rc = setup_fwd_kernel(kern, C::SMEM_BYTES, checked))) return rc;
+  const long long grid = items;
   kern<<<(unsigned)grid, R::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   TATTN_CUDA(cudaGetLastError());
   return ATTN_OK;
