@@ -39,7 +39,8 @@ from attn_workloads import (APB_WORKLOADS, DECODE_WORKLOADS, WORKLOADS, decode_b
 
 
 KERNEL_SOURCES = ("tiled_attention_22_b200/csrc/attn_fwd_kernels.cuh", "tiled_attention_22_b200/csrc/ptx.cuh",
-                  "tiled_attention_22_b200/csrc/attn_fwd_launch.cuh", "tiled_attention_22_b200/csrc/tma_host.cuh")
+                  "tiled_attention_22_b200/csrc/attn_fwd_launch.cuh", "tiled_attention_22_b200/csrc/tma_host.cuh",
+                  "tiled_attention_22_b200/csrc/attn_fwd_persistent.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_kernel_traffic_mha_causal_b4_h32_n4096_d128.txt")
 
 
