@@ -553,7 +553,7 @@ def run_context_parallel(args, dev, world, peaks, ranks=4):
     out = {w.name + f"_ring{ranks}": {
         "ms_per_call": res["ring"], "TFLOP/s": tf * world, "frac_of_bf16_peak": tf / peaks["bf16_sustained"],
         "single_call_ms": res["single_call"], "ring_over_single": res["ring"] / res["single_call"],
-        "launches_per_call": 2 * steps, "kernels": "attn_fwd_kernel<128,bf16> + lse_merge_kernel<128,bf16>",
+        "launches_per_call": 2 * steps, "kernels": "attn_fwd_persistent_kernel<128,bf16> + lse_merge_kernel<128,bf16>",
         "note": "all ranks' steps on one GPU; the key/value exchange over NVLink is not timed"}}
     out["peak_note"] = "bf16 dense GEMM %.0f TFLOP/s (%s, sustained)" % (peaks["bf16_sustained"], peaks["source"])
     del q, k, v, qs, kv, o
