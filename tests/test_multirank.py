@@ -34,7 +34,7 @@ def _rank_main(rank, world, port, out):
 @pytest.mark.timeout(120)
 def test_two_gloo_ranks_aggregate_max_time_and_total_work():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
     for rank in range(world):
         ms, tflops = out[rank]

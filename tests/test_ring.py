@@ -4,6 +4,7 @@ NCCL.  The attention arithmetic of each step is checked on the GPU (test_gpu_rin
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -73,7 +74,7 @@ def _rank_main(rank, world, port, out):
 @pytest.mark.timeout(180)
 @pytest.mark.parametrize("world", [2, 3])
 def test_gloo_ring_delivers_block_r_minus_s(world):
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
     for r in range(world):
         res, untouched = out[r]
@@ -82,3 +83,55 @@ def test_gloo_ring_delivers_block_r_minus_s(world):
         for s, j, k_ok, v_ok in res:
             assert j == (r - s) % world
             assert k_ok and v_ok, f"rank {r} step {s}: block {j} arrived wrong"
+
+
+def _join(Oa, La, Ob, Lb):
+    """The log-sum-exp join of two partial attention results (float64)."""
+    m = np.maximum(La, Lb)
+    safe = np.where(np.isneginf(m), 0.0, m)
+    wa, wb = np.exp(La - safe), np.exp(Lb - safe)
+    s = wa + wb
+    with np.errstate(invalid="ignore", divide="ignore"):
+        O = (wa[..., None] * Oa + wb[..., None] * Ob) / s[..., None]
+        L = safe + np.log(s)
+    return np.where(np.isneginf(m)[..., None], 0.0, O), np.where(np.isneginf(m), -np.inf, L)
+
+
+@pytest.mark.parametrize("split", [1, 37, 64, 99])
+def test_partials_over_key_blocks_join_to_full_attention(split):
+    """Ring attention's premise: attention over keys A u B is the log-sum-exp join of the attention
+    over A and over B (which pins the oracle's lse as well: a wrong lse breaks the join)."""
+    import oracle
+    from attn_workloads import Workload, make_inputs
+
+    w = Workload("j", 1, 4, 2, 100, 64, False, "bf16", "k_offset", 4242)
+    q, k, v = make_inputs(w)
+    O, L = oracle.attention(q, k, v, w.scale, False)
+    Oa, La = oracle.attention(q, k[:, :, :split], v[:, :, :split], w.scale, False)
+    Ob, Lb = oracle.attention(q, k[:, :, split:], v[:, :, split:], w.scale, False)
+    Oj, Lj = _join(Oa, La, Ob, Lb)
+    np.testing.assert_allclose(Oj, O, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Lj, L, rtol=0, atol=1e-12)
+
+
+def test_causal_ring_blocks_join_to_causal_attention():
+    """The causal ring over 4 blocks: rank r joins its diagonal block (causal within the block) and
+    the full blocks before it, and gets the rows of causal attention over the whole sequence."""
+    import oracle
+    from attn_workloads import Workload, make_inputs
+
+    W, n = 4, 40
+    w = Workload("c", 1, 2, 1, W * n, 64, True, "bf16", "normal", 4343)
+    q, k, v = make_inputs(w)
+    O, L = oracle.attention(q, k, v, w.scale, True)
+    for r in range(W):
+        qr = q[:, :, r * n:(r + 1) * n]
+        acc = None
+        for s, j, kind in ring_schedule(r, W, True):
+            if kind == "skip":
+                continue
+            kj, vj = k[:, :, j * n:(j + 1) * n], v[:, :, j * n:(j + 1) * n]
+            part = oracle.attention(qr, kj, vj, w.scale, kind == "causal")
+            acc = part if acc is None else _join(acc[0], acc[1], part[0], part[1])
+        np.testing.assert_allclose(acc[0], O[:, :, r * n:(r + 1) * n], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(acc[1], L[:, :, r * n:(r + 1) * n], rtol=0, atol=1e-12)
