@@ -80,6 +80,17 @@ enum attn_dtype { ATTN_BF16 = 0, ATTN_FP16 = 1 };
  *   workspace / ws_bytes: device memory of at least
  *     attn_workspace_bytes(B,Hq,Hkv,N,d,mode) bytes (0 for BF16_EXACT, where
  *     workspace may be NULL).  Its content on entry does not matter.
+ *   Launches: BF16_EXACT with d = 128 runs on persistent CTAs (one per SM)
+ *     that take 256-row work items from a counter inside the library, one
+ *     counter per stream handle (256 per device; calls from further streams
+ *     take one CTA per item, with the same results), cleared by a 4-byte
+ *     cudaMemsetAsync on the stream before the kernel.  Calls on one stream are
+ *     ordered by the stream and calls on different streams use different
+ *     counters; a stream handle destroyed while its call still runs must not
+ *     be reused by a new stream that calls this function before that call
+ *     ends.  The first call on a device looks up the counters' address (with
+ *     that device current): make it before any stream capture on the device.
+ *     The other modes and d = 64 launch one CTA per work item.
  */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int d, int causal, float scale, int mode,
