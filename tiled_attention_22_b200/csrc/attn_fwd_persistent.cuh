@@ -73,12 +73,12 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int idx) {
 }
 
 // Persistent CTAs (one per SM): warp 11 takes work items from a global ticket counter (cleared
-// before the launch) and hands them to the other roles through a ring of ITEM_RING shared-memory
-// slots, so items go to CTAs in order, as they free up, and one CTA's set-up, TMEM allocation and
-// first loads serve many items.  Across items the roles keep their ring
-// positions and barrier phases; the next item's Q is loaded (warp 10) as soon as the MMAs of the
-// previous item no longer read that query tile's buffer, and its first Q K^T is issued right
-// after the previous item's last P V, while the softmax warps still write out the previous O.
+// before the launch) and hands them, decoded, to the other roles through a ring of ITEM_RING
+// shared-memory slots, so items go to CTAs in order, as they free up, and one CTA's set-up, TMEM
+// allocation and first loads serve many items.  Across items the roles keep their ring positions
+// and barrier phases; the next item's Q is loaded (warp 10) as soon as the MMAs of the previous
+// item no longer read that query tile's buffer, and its first Q K^T is issued right after the
+// previous item's last P V, while the softmax warps still write out the previous O.
 template <int D, int QK, bool FP16>
 __global__ void __launch_bounds__(FwdRoles<false>::kThreads, 1)
     attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
