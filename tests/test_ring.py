@@ -135,3 +135,29 @@ def test_causal_ring_blocks_join_to_causal_attention():
             acc = part if acc is None else _join(acc[0], acc[1], part[0], part[1])
         np.testing.assert_allclose(acc[0], O[:, :, r * n:(r + 1) * n], rtol=0, atol=1e-12)
         np.testing.assert_allclose(acc[1], L[:, :, r * n:(r + 1) * n], rtol=0, atol=1e-12)
+
+
+def test_emulated_ring_needs_a_divisible_sequence():
+    from tiled_attention_22_b200.ring import ring_attention_emulated
+
+    q = torch.zeros(1, 2, 10, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="multiple"):
+        ring_attention_emulated(q, q[:, :1], q[:, :1], 3)
+
+
+def test_merge_binding_validates_arguments_on_the_host():
+    """attn_merge_lse checks shapes, dtypes and devices before it reaches the library."""
+    from tiled_attention_22_b200 import attn_merge_lse
+
+    acc = torch.zeros(4, 128)
+    lacc = torch.zeros(4)
+    part = torch.zeros(4, 128, dtype=torch.bfloat16)
+    lp = torch.zeros(4)
+    with pytest.raises(ValueError):  # float32 accumulator required
+        attn_merge_lse(acc.double(), lacc, part, lp)
+    with pytest.raises(ValueError):  # one lse per row
+        attn_merge_lse(acc, torch.zeros(5), part, lp)
+    with pytest.raises(ValueError):  # nothing to merge and nowhere to write
+        attn_merge_lse(acc, lacc)
+    with pytest.raises(ValueError):  # CUDA tensors only
+        attn_merge_lse(acc, lacc, part, lp)
