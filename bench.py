@@ -1,15 +1,18 @@
 #!/usr/bin/env python
 """Benchmark of the tiled attention forward pass on B200.
 
-One step = one pass of the whole hot path over the headline workload
-(B=4, H=32, N=4096, d=128, causal, bf16; scale 1/sqrt(128)) in int8_qk mode:
-K-mean / smoothing / INT8 quantisation pre-pass, then the fused INT8-QK^T /
-16-bit-PV attention kernel.  bf16_exact is timed the same way and reported
-under "modes".  Metric: attention FLOPs 4*B*H*N^2*d/2 per step over device
-time (TFLOP/s), whole job (sum over ranks / max time over ranks).
+One step = one pass of the whole hot path over the headline workload, the largest single-GPU one
+(B=1, Hq=32, Hkv=8, N=131072, d=128, causal, bf16, K with per-channel offsets; scale 1/sqrt(128))
+in int8_qk mode: K-mean / smoothing / INT8 quantisation pre-pass, then the fused INT8-QK^T /
+16-bit-PV attention kernel.  bf16_exact and fp8_qk are timed the same way under "modes", and the
+other workloads at N >= 4096 under "other_configs".  Metric: attention FLOPs 4*B*Hq*N^2*d/2 per
+step over device time (TFLOP/s), whole job (sum over ranks / max time over ranks).  Each mode's
+fused kernel is also reported as a fraction of its own dense tensor peak (bf16 for bf16_exact,
+INT8 for int8_qk, FP8 for fp8_qk), with the mixed peak (Q K^T at the 8-bit rate, P V at the bf16
+rate) beside it as the explanation.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                  [--config 2] [--no-e2e] [--no-cpu-baseline]
+                  [--config 5] [--no-e2e] [--no-cpu-baseline] [--no-decode] [--no-others]
 
 Multi-GPU: one process per GPU (torchrun); each rank runs its own independent
 batch of the workload (the (batch, head) units share nothing), so no
@@ -41,7 +44,12 @@ from attn_workloads import (APB_WORKLOADS, DECODE_WORKLOADS, WORKLOADS, decode_b
 KERNEL_SOURCES = ("tiled_attention_22_b200/csrc/attn_fwd_kernels.cuh", "tiled_attention_22_b200/csrc/ptx.cuh",
                   "tiled_attention_22_b200/csrc/attn_fwd_launch.cuh", "tiled_attention_22_b200/csrc/tma_host.cuh",
                   "tiled_attention_22_b200/csrc/attn_fwd_persistent.cuh")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_kernel_traffic_mha_causal_b4_h32_n4096_d128.txt")
+
+# A fused-kernel launch at least this long is a sustained load in its own right (75x the 0.67 ms
+# calls of the burst GEMM measurement); its fraction of peak uses the sustained bf16 rate when the
+# clock record of the timed region also shows the power cap acting.  Shorter launches use the
+# burst rate.  Both fractions are always reported.
+LONG_LAUNCH_MS = 50.0
 
 
 def _kernel_source_hash():
@@ -54,13 +62,19 @@ def _kernel_source_hash():
     return h.hexdigest()
 
 
-def _measured_traffic(mode):
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary, or None when the
-    kernel sources changed since those counters were taken (or no summary exists)."""
-    if not os.path.exists(TRAFFIC_FILE):
+def _traffic_file(workload_name):
+    return os.path.join(ROOT, "profiles", f"attn_fwd_traffic_{workload_name}.txt")
+
+
+def _measured_traffic(workload_name, mode):
+    """DRAM bytes per launch of the mode's fused kernel on this workload, from the committed ncu
+    summary, or None when the kernel sources changed since those counters were taken (or no
+    summary exists)."""
+    path = _traffic_file(workload_name)
+    if not os.path.exists(path):
         return None
     fields = {}
-    with open(TRAFFIC_FILE) as f:
+    with open(path) as f:
         for line in f:
             if "=" in line and not line.lstrip().startswith("#"):
                 key, val = line.split("=", 1)
@@ -68,7 +82,7 @@ def _measured_traffic(mode):
     if fields.get("kernel_source_sha256") != _kernel_source_hash():
         return None
     val = fields.get(f"{mode}_dram_bytes_per_launch")
-    return int(val) if val else None
+    return int(float(val)) if val else None
 
 
 def _peaks():
@@ -79,6 +93,40 @@ def _peaks():
         return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
                 "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def _gemm_peaks(dev):
+    """Dense 8-bit GEMM rates on this GPU, measured here as alternative denominators (library GEMMs,
+    timing only): torch._int_mm (INT8 -> int32) and torch._scaled_mm (E4M3 -> bf16) at 8192^3,
+    best of 10 after warm-up, CUDA events."""
+    n = 8192
+    out = {}
+    try:
+        a = torch.randint(-127, 128, (n, n), device=dev, dtype=torch.int8)
+        b = torch.randint(-127, 128, (n, n), device=dev, dtype=torch.int8).t()
+        fa = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        fb = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev)
+        fns = {"int8_tops": lambda: torch._int_mm(a, b),
+               "fp8_tflops": lambda: torch._scaled_mm(fa, fb, one, one, out_dtype=torch.bfloat16)}
+        for name, fn in fns.items():
+            for _ in range(3):
+                fn()
+            best = float("inf")
+            for _ in range(10):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                best = min(best, e0.elapsed_time(e1))
+            out[name] = 2.0 * n ** 3 / (best * 1e-3) / 1e12
+        del a, b, fa, fb
+        torch.cuda.empty_cache()
+    except (RuntimeError, AttributeError) as e:  # timing only; the headline does not depend on it
+        out["error"] = str(e).splitlines()[0][:120]
+    out["how"] = "torch._int_mm / torch._scaled_mm 8192^3, best of 10"
+    return out
 
 
 class ClockSampler:
@@ -185,36 +233,56 @@ def whole_job_rate(local_ms, flops_per_rank, world, device="cuda"):
     return ms, flops_per_rank * world / (ms * 1e-3) / 1e12
 
 
-def cpu_baseline(w, budget_s=15.0):
-    """The CPU oracle (float64 numpy, as it stands) on a bounded sample of the workload: the int8
-    emulation pre-pass and the attention of whole heads, as many heads as fit in the budget."""
+def _oracle_sample(w, q, k, v, units, rows_per_unit, budget_s=None):
+    """The CPU oracle (float64 numpy, as it stands) on a sample of the workload: for each sampled
+    (batch, query head) unit, the INT8 emulation pre-pass of that head (its Q head and kv head)
+    and the dequantised float64 attention of ``rows_per_unit`` query rows spread over the sequence.
+    The oracle computes every row against all N keys (masked), so its cost per row does not depend
+    on the row's position; the whole workload's time is extrapolated as
+    units_total * (pre-pass time per unit + row time per row * N).  Returns (TFLOP/s, seconds
+    spent, description)."""
     import numpy as np
 
     import oracle
 
-    cores = len(os.sched_getaffinity(0))
-    q, k, v = make_inputs(w)
     G = w.Hq // w.Hkv
-    t0 = time.perf_counter()
-    flops = 0.0
-    heads = 0
-    for b in range(w.B):
-        for h in range(w.Hq):
-            g = h // G
-            qs, ks, vs = q[b:b + 1, h:h + 1], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1]
-            q8, sq, k8, sk, mean, bias = oracle.prepass(qs, ks, w.scale)
-            oracle.attention_int8(q8, sq, k8, sk, bias, vs, w.scale, w.causal)
-            flops += 4.0 * w.N * w.N * w.d / (2.0 if w.causal else 1.0)
-            heads += 1
-            if time.perf_counter() - t0 > budget_s:
-                break
-        if time.perf_counter() - t0 > budget_s:
+    all_units = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    rng = np.random.default_rng(w.seed_base + 17)
+    order = rng.permutation(len(all_units))
+    rows = np.unique(np.linspace(0, w.N - 1, rows_per_unit).astype(np.int64))
+    t_pre = t_rows = 0.0
+    done = 0
+    t_start = time.perf_counter()
+    for idx in order[:units]:
+        b, h = all_units[idx]
+        g = h // G
+        qs, ks, vs = q[b:b + 1, h:h + 1], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1]
+        t0 = time.perf_counter()
+        q8, sq, k8, sk, mean, bias = oracle.prepass(qs, ks, w.scale)
+        t1 = time.perf_counter()
+        oracle.attention_int8(q8, sq, k8, sk, bias, vs, w.scale, w.causal, rows=rows)
+        t2 = time.perf_counter()
+        t_pre += t1 - t0
+        t_rows += t2 - t1
+        done += 1
+        if budget_s is not None and time.perf_counter() - t_start > budget_s:
             break
-    dt = time.perf_counter() - t0
-    del np
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{heads} of {w.B * w.Hq} (batch, head) units, all {w.N} rows each: INT8 emulation "
-                      f"pre-pass + float64 attention, {dt:.1f} s", "seconds": dt}
+    per_unit = t_pre / done + t_rows / (done * len(rows)) * w.N
+    total_s = per_unit * len(all_units)
+    value = w.flops() / total_s / 1e12
+    desc = (f"{done} of {len(all_units)} (batch, head) units x {len(rows)} query rows spread over N={w.N}: "
+            f"INT8 emulation pre-pass of the unit's heads + dequantised float64 attention of those rows, "
+            f"{t_pre + t_rows:.1f} s; extrapolated to the whole workload as units x (pre-pass + "
+            f"row time x N) = {total_s:.3g} s")
+    return value, t_pre + t_rows, desc
+
+
+def cpu_baseline(w, q, k, v, budget_s=15.0):
+    """The oracle timed on the host cores on a bounded sample of the headline workload."""
+    cores = len(os.sched_getaffinity(0))
+    value, spent, desc = _oracle_sample(w, q, k, v, units=w.B * w.Hq, rows_per_unit=48, budget_s=budget_s)
+    return {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc, "seconds": spent,
+            "extrapolated": True}
 
 
 def run_reference(args, w, world, rank):
@@ -223,40 +291,144 @@ def run_reference(args, w, world, rank):
             "warmup": args.warmup}
     if rank != 0:
         return None
-    import oracle
-
     q, k, v = make_inputs(w)
-    G = w.Hq // w.Hkv
-    per_step_heads = 1
-    total_flops = 0.0
-    t_total = 0.0
-    idx = 0
+    rows = 16
+    vals, t_total = [], 0.0
     for step in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        flops = 0.0
-        for _ in range(per_step_heads):
-            b, h = divmod(idx % (w.B * w.Hq), w.Hq)
-            idx += 1
-            g = h // G
-            qs, ks, vs = q[b:b + 1, h:h + 1], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1]
-            q8, sq, k8, sk, mean, bias = oracle.prepass(qs, ks, w.scale)
-            oracle.attention_int8(q8, sq, k8, sk, bias, vs, w.scale, w.causal)
-            flops += 4.0 * w.N * w.N * w.d / (2.0 if w.causal else 1.0)
-        dt = time.perf_counter() - t0
+        value, spent, desc = _oracle_sample(w, q, k, v, units=1, rows_per_unit=rows)
         if step >= args.warmup:
-            total_flops += flops
-            t_total += dt
-    value = total_flops / t_total / 1e12
+            vals.append(value)
+            t_total += spent
+    value = statistics.mean(vals)
     cores = len(os.sched_getaffinity(0))
     line.update({"value": value, "ms_per_step": 1e3 * t_total / args.steps, "scaling": "weak",
                  "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                  "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
                             "causal": w.causal},
                  "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                  "sample": f"each step: {per_step_heads} (batch, head) unit of the workload, "
-                                            f"all {w.N} rows, INT8 emulation pre-pass + float64 attention"},
+                                  "sample": f"each step: {desc}"},
                  "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
     return line
+
+
+class _Modes:
+    """Device buffers of one workload and the step of each mode (pre-pass and fused kernel
+    separately timed with CUDA events on the launching stream)."""
+
+    def __init__(self, ta, w, q, k, v, dev):
+        self.ta, self.w = ta, w
+        B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+        self.qd, self.kd, self.vd = q.to(dev), k.to(dev), v.to(dev)
+        self.o = torch.empty_like(self.qd)
+        self.lse = torch.empty((B, Hq, N), device=dev, dtype=torch.float32)
+        T = (N + 127) // 128
+        self.pre = dict(q8=torch.empty((B, Hq, N, d), device=dev, dtype=torch.int8),
+                        sq=torch.empty((B, Hq, T), device=dev, dtype=torch.float32),
+                        k8=torch.empty((B, Hkv, N, d), device=dev, dtype=torch.int8),
+                        sk=torch.empty((B, Hkv, T), device=dev, dtype=torch.float32),
+                        kmean=torch.empty((B, Hkv, d), device=dev, dtype=torch.float32),
+                        lse_bias=torch.empty((B, Hq, N), device=dev, dtype=torch.float32))
+        self.pre8 = dict(self.pre, q8=self.pre["q8"].view(torch.uint8), k8=self.pre["k8"].view(torch.uint8))
+        self.scratch = torch.empty(ta.attn_quant_scratch_bytes(B, Hkv, N, d), device=dev, dtype=torch.uint8)
+        self.stream = torch.cuda.current_stream()
+        self.steps = {"int8_qk": (self.step_int8, 2), "bf16_exact": (self.step_bf16, 1),
+                      "fp8_qk": (self.step_fp8, 2)}
+
+    def step_int8(self, ev=None):
+        ta, w, s = self.ta, self.w, self.stream
+        if ev:
+            ev[0].record(s)
+        ta.attn_quant_smooth_k(self.qd, self.kd, scale=w.scale, scratch=self.scratch, stream=s, out=self.pre)
+        if ev:
+            ev[1].record(s)
+        ta.attn_fwd_int8_quantized(self.pre, self.vd, causal=w.causal, scale=w.scale, out=self.o, lse=self.lse,
+                                   stream=s)
+        if ev:
+            ev[2].record(s)
+
+    def step_fp8(self, ev=None):
+        ta, w, s = self.ta, self.w, self.stream
+        if ev:
+            ev[0].record(s)
+        ta.attn_quant_smooth_k_fp8(self.qd, self.kd, scale=w.scale, scratch=self.scratch, stream=s, out=self.pre8)
+        if ev:
+            ev[1].record(s)
+        ta.attn_fwd_fp8_quantized(self.pre8, self.vd, causal=w.causal, scale=w.scale, out=self.o, lse=self.lse,
+                                  stream=s)
+        if ev:
+            ev[2].record(s)
+
+    def step_bf16(self, ev=None):
+        ta, w, s = self.ta, self.w, self.stream
+        if ev:
+            ev[0].record(s)
+        ta.attn_fwd(self.qd, self.kd, self.vd, causal=w.causal, scale=w.scale, mode="bf16_exact", out=self.o,
+                    lse=self.lse, stream=s)
+        if ev:
+            ev[1].record(s)
+
+    def time(self, mode, steps, warmup, world, sampler=None):
+        fn, nk = self.steps[mode]
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        _barrier(world)
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(steps)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if sampler is not None:
+            sampler.mark("t0")
+        start.record(self.stream)
+        for st in range(steps):
+            fn(evs[st])
+        end.record(self.stream)
+        torch.cuda.synchronize()
+        if sampler is not None:
+            sampler.mark("t1")
+        _barrier(world)
+        torch.cuda.synchronize()
+        ms, tflops = whole_job_rate(start.elapsed_time(end), self.w.flops() * steps, world)
+        if self.ta.attn_check_status() != 0:
+            raise RuntimeError("device-side wait timed out during the benchmark")
+        kern = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(nk)]
+        return {"ms_total": ms, "ms_per_step": ms / steps, "tflops": tflops, "kernel_ms": kern}
+
+
+def _bf16_peak(peaks, launch_ms, clocks):
+    """(peak TFLOP/s, 'burst'|'sustained') for a fused-kernel launch of this duration."""
+    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+    if launch_ms >= LONG_LAUNCH_MS and capped:
+        return peaks["bf16_sustained"], "sustained"
+    return peaks["bf16"], "burst"
+
+
+def _mode_report(w, mode, r, peaks, clocks, gemm):
+    """Per-mode figures: step and fused-kernel TFLOP/s, and the fused kernel against its own dense
+    peak (bf16 / INT8 / FP8 = 2 x bf16 by the nominal ratio), the mixed peak, and both burst and
+    sustained bf16 bases."""
+    flops = w.flops()
+    fused_ms = r["kernel_ms"][-1]
+    fused = flops / (fused_ms * 1e-3) / 1e12
+    bf16, basis = _bf16_peak(peaks, fused_ms, clocks)
+    out = {"tflops": r["tflops"], "ms_per_step": r["ms_per_step"], "fused_ms": fused_ms, "fused_tflops": fused,
+           "peak_basis": basis}
+    if mode == "bf16_exact":
+        out["frac_of_bf16_peak"] = fused / bf16
+        out["frac_of_bf16_burst"] = fused / peaks["bf16"]
+        out["frac_of_bf16_sustained"] = fused / peaks["bf16_sustained"]
+        return out
+    key = "int8" if mode == "int8_qk" else "fp8"
+    out["prepass_ms"] = r["kernel_ms"][0]
+    out["prepass_gbs"] = _prepass_bytes(w) / (r["kernel_ms"][0] * 1e-3) / 1e9
+    out["prepass_frac_of_hbm_peak"] = out["prepass_gbs"] / peaks["hbm_gbs"]
+    out[f"frac_of_{key}_peak"] = fused / (2.0 * bf16)
+    out[f"frac_of_{key}_burst"] = fused / (2.0 * peaks["bf16"])
+    out[f"frac_of_{key}_sustained"] = fused / (2.0 * peaks["bf16_sustained"])
+    out["frac_of_mixed_peak"] = fused / (bf16 * 4.0 / 3.0)
+    alt = gemm.get("int8_tops" if key == "int8" else "fp8_tflops")
+    if alt:
+        out[f"frac_of_measured_{key}_gemm"] = fused / alt
+    return out
 
 
 def run_native(args, w, world, rank, local):
@@ -264,81 +436,21 @@ def run_native(args, w, world, rank, local):
 
     dev = torch.device("cuda", local)
     q, k, v = make_inputs(w)
-    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
-    o = torch.empty_like(qd)
-    lse = torch.empty((B, Hq, N), device=dev, dtype=torch.float32)
-    T = (N + 127) // 128
-    pre = dict(q8=torch.empty((B, Hq, N, d), device=dev, dtype=torch.int8),
-               sq=torch.empty((B, Hq, T), device=dev, dtype=torch.float32),
-               k8=torch.empty((B, Hkv, N, d), device=dev, dtype=torch.int8),
-               sk=torch.empty((B, Hkv, T), device=dev, dtype=torch.float32),
-               kmean=torch.empty((B, Hkv, d), device=dev, dtype=torch.float32),
-               lse_bias=torch.empty((B, Hq, N), device=dev, dtype=torch.float32))
-    scratch = torch.empty(ta.attn_quant_scratch_bytes(B, Hkv, N, d), device=dev, dtype=torch.uint8)
-    pre8 = dict(pre, q8=pre["q8"].view(torch.uint8), k8=pre["k8"].view(torch.uint8))
-    stream = torch.cuda.current_stream()
-    flops = w.flops()
+    modes = [m for m in ("int8_qk", "bf16_exact", "fp8_qk") if m in args.modes.split(",")]
+    peaks = _peaks()
+    gemm = _gemm_peaks(dev) if not args.no_gemm_peaks else {}
 
-    def step_int8(ev=None):
-        if ev:
-            ev[0].record(stream)
-        ta.attn_quant_smooth_k(qd, kd, scale=w.scale, scratch=scratch, stream=stream, out=pre)
-        if ev:
-            ev[1].record(stream)
-        ta.attn_fwd_int8_quantized(pre, vd, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
-        if ev:
-            ev[2].record(stream)
-
-    def step_fp8(ev=None):
-        if ev:
-            ev[0].record(stream)
-        ta.attn_quant_smooth_k_fp8(qd, kd, scale=w.scale, scratch=scratch, stream=stream, out=pre8)
-        if ev:
-            ev[1].record(stream)
-        ta.attn_fwd_fp8_quantized(pre8, vd, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
-        if ev:
-            ev[2].record(stream)
-
-    def step_bf16(ev=None):
-        if ev:
-            ev[0].record(stream)
-        ta.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, mode="bf16_exact", out=o, lse=lse, stream=stream)
-        if ev:
-            ev[1].record(stream)
-
+    mb = _Modes(ta, w, q, k, v, dev)
     results = {}
     sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
                            if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local)
     sampler.start()
     time.sleep(0.3)
-    for mode, fn, nk in (("int8_qk", step_int8, 2), ("bf16_exact", step_bf16, 1), ("fp8_qk", step_fp8, 2)):
-        if mode not in args.modes.split(","):
-            continue
-        for _ in range(args.warmup):
-            fn()
-        torch.cuda.synchronize()
-        _barrier(world)
-        torch.cuda.synchronize()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
-        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if mode == "int8_qk":
-            sampler.mark("t0")
-        start.record(stream)
-        for s in range(args.steps):
-            fn(evs[s])
-        end.record(stream)
-        torch.cuda.synchronize()
-        if mode == "int8_qk":
-            sampler.mark("t1")
-        _barrier(world)
-        torch.cuda.synchronize()
-        ms, tflops = whole_job_rate(start.elapsed_time(end), flops * args.steps, world)
-        if ta.attn_check_status() != 0:
-            raise RuntimeError("device-side wait timed out during the benchmark")
-        kern = [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i in range(nk)]
-        results[mode] = {"ms_total": ms, "ms_per_step": ms / args.steps, "tflops": tflops, "kernel_ms": kern}
+    for mode in modes:
+        results[mode] = mb.time(mode, args.steps, args.warmup, world, sampler if mode == "int8_qk" else None)
     clocks = sampler.stop()
+    o, lse = mb.o, mb.lse
 
     # end to end through the public C ABI with host buffers: H2D q,k,v + forward + D2H o, lse
     e2e = None
@@ -349,76 +461,90 @@ def run_native(args, w, world, rank, local):
         ws = torch.empty(ta.attn_workspace_bytes(B, Hq, Hkv, N, d, "int8_qk"), device=dev, dtype=torch.uint8)
         e_steps = max(3, min(args.steps, 50))
         for _ in range(2):
-            ta.attn_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, causal=w.causal, scale=w.scale,
-                             mode="int8_qk", workspace=ws, stream=stream)
+            ta.attn_fwd_host(qh, kh, vh, oh, lh, mb.qd, mb.kd, mb.vd, o, lse, causal=w.causal, scale=w.scale,
+                             mode="int8_qk", workspace=ws, stream=mb.stream)
         _barrier(world)
         torch.cuda.synchronize()
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
+        s0.record(mb.stream)
         for _ in range(e_steps):
-            ta.attn_fwd_host(qh, kh, vh, oh, lh, qd, kd, vd, o, lse, causal=w.causal, scale=w.scale,
-                             mode="int8_qk", workspace=ws, stream=stream)
-        s1.record(stream)
+            ta.attn_fwd_host(qh, kh, vh, oh, lh, mb.qd, mb.kd, mb.vd, o, lse, causal=w.causal, scale=w.scale,
+                             mode="int8_qk", workspace=ws, stream=mb.stream)
+        s1.record(mb.stream)
         torch.cuda.synchronize()
-        ems, e2e_tflops = whole_job_rate(s0.elapsed_time(s1), flops * e_steps, world)
+        ems, e2e_tflops = whole_job_rate(s0.elapsed_time(s1), w.flops() * e_steps, world)
         e2e = {"value": e2e_tflops, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(3 * q.numel() * q.element_size()),
                "d2h_bytes_per_step": int(o.numel() * o.element_size() + lse.numel() * 4),
                "steps": e_steps, "ms_per_step": ems / e_steps}
+        del qh, kh, vh, oh, lh, ws
+    del mb
+    torch.cuda.empty_cache()
 
-    peaks = _peaks()
     nan = {"ms_total": float("nan"), "ms_per_step": float("nan"), "tflops": float("nan"),
            "kernel_ms": [float("nan"), float("nan")]}
-    r8 = results.get("int8_qk", nan)
-    rb = results.get("bf16_exact", nan)
-    rf = results.get("fp8_qk", nan)
-    long_region = r8["ms_total"] > 1000.0
-    bf16_peak = peaks["bf16_sustained"] if long_region else peaks["bf16"]
-    mixed_peak = bf16_peak * 4.0 / 3.0  # QK^T at the INT8 rate (2x bf16, nominal ratio), PV at the bf16 rate
-    fused_ms = r8["kernel_ms"][1]
-    achieved = flops / (fused_ms * 1e-3) / 1e12
+    rep = {m: _mode_report(w, m, results.get(m, nan), peaks, clocks, gemm) for m in modes}
+    r8 = rep["int8_qk"] if "int8_qk" in rep else _mode_report(w, "int8_qk", nan, peaks, clocks, gemm)
+    bf16_peak, basis = _bf16_peak(peaks, r8["fused_ms"], clocks)
+    int8_peak = 2.0 * bf16_peak
+    achieved = r8["fused_tflops"]
+    alt = gemm.get("int8_tops")
     line = {
         "metric": f"attention fwd TFLOP/s (int8_qk step) on {w.name}",
-        "value": r8["tflops"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": r8["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8", "data": "synthetic",
+        "value": results.get("int8_qk", nan)["tflops"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": results.get("int8_qk", nan)["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
                    "causal": w.causal, "input_dtype": w.dtype, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (q, k, v = %.0f MB per rank)" % (3 * q.numel() * 2 / 1e6)},
-        "modes": {
-            "int8_qk": {"tflops": r8["tflops"], "ms_per_step": r8["ms_per_step"],
-                        "prepass_ms": r8["kernel_ms"][0], "fused_ms": fused_ms,
-                        "fused_tflops": achieved,
-                        "prepass_gbs": _prepass_bytes(w) / (r8["kernel_ms"][0] * 1e-3) / 1e9,
-                        "prepass_frac_of_hbm_peak": _prepass_bytes(w) / (r8["kernel_ms"][0] * 1e-3) / 1e9
-                        / peaks["hbm_gbs"]},
-            "fp8_qk": {"tflops": rf["tflops"], "ms_per_step": rf["ms_per_step"],
-                       "prepass_ms": rf["kernel_ms"][0], "fused_ms": rf["kernel_ms"][1],
-                       "fused_tflops": flops / (rf["kernel_ms"][1] * 1e-3) / 1e12,
-                       "frac_of_mixed_peak": (flops / (rf["kernel_ms"][1] * 1e-3) / 1e12) / mixed_peak},
-            "bf16_exact": {"tflops": rb["tflops"], "ms_per_step": rb["ms_per_step"],
-                           "frac_of_bf16_peak": (flops / (rb["kernel_ms"][0] * 1e-3) / 1e12) / bf16_peak,
-                           "traffic": _measured_traffic("bf16_exact"),
-                           "algorithmic_bytes": _fused_bytes(w, "bf16_exact")},
-        },
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": mixed_peak, "unit": "TFLOP/s",
-                     "frac": achieved / mixed_peak, "traffic": _measured_traffic("int8_qk"),
+                   "l2": "inputs larger than L2 (q, k, v = %.0f MB per rank)" % (
+                       (q.numel() + k.numel() + v.numel()) * 2 / 1e6)},
+        "modes": rep,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
+                     "frac": achieved / int8_peak, "traffic": _measured_traffic(w.name, "int8_qk"),
                      "algorithmic_bytes": _fused_bytes(w, "int8_qk"),
                      "kernel": "attn_fwd_kernel<128,int8,bf16>",
-                     "peak_note": ("4/3 x measured bf16 %s (%s): INT8 half of the FLOPs at 2x the bf16 rate"
-                                   % ("sustained" if long_region else "burst", peaks["source"]))},
+                     "peak_note": ("INT8 dense = 2 x measured bf16 %s (%s; nominal INT8/bf16 ratio 4.5/2.25 "
+                                   "PFLOP/s); mixed peak 4/3 x bf16 gives frac %.3f; the INT8 GEMM measured "
+                                   "here (torch._int_mm) %s"
+                                   % (basis, peaks["source"], achieved / (bf16_peak * 4.0 / 3.0),
+                                      ("%.1f TOPS gives frac %.3f" % (alt, achieved / alt)) if alt
+                                      else "was not measured"))},
+        "gemm_peaks_measured_here": gemm,
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
     if e2e:
         line["e2e"] = e2e
+    if not args.no_others:
+        line["other_configs"] = run_other_configs(args, ta, dev, world, peaks, gemm, skip=w)
     if not args.no_decode:
         line["decode"] = run_decode(args, dev, world, peaks)
         line["prefix_mask"] = run_prefix_mask(args, dev, world, peaks)
-        line["context_parallel"] = run_context_parallel(args, dev, world, peaks)
+        line["context_parallel"] = run_context_parallel(args, dev, world, peaks,
+                                                        inputs=(q, k, v) if w is WORKLOADS[5] else None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"] = cpu_baseline(w, q, k, v)
     return line
+
+
+def run_other_configs(args, ta, dev, world, peaks, gemm, skip=None):
+    """The other workloads at N >= 4096 (4096-token MHA, the 8192-token GQA, the 16384-token d = 64
+    one): every mode, the same steps, with the same per-mode figures as the headline."""
+    out = {}
+    modes = [m for m in ("int8_qk", "bf16_exact", "fp8_qk") if m in args.modes.split(",")]
+    for cfg in (2, 3, 4):
+        w = WORKLOADS[cfg]
+        if w is skip:
+            continue
+        q, k, v = make_inputs(w)
+        mb = _Modes(ta, w, q, k, v, dev)
+        res = {}
+        for mode in modes:
+            res[mode] = mb.time(mode, args.steps, args.warmup, world)
+        out[w.name] = {m: _mode_report(w, m, res[m], peaks, None, gemm) for m in modes}
+        del mb
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_decode(args, dev, world, peaks):
@@ -507,16 +633,18 @@ def run_prefix_mask(args, dev, world, peaks):
     return out
 
 
-def run_context_parallel(args, dev, world, peaks, ranks=4):
+def run_context_parallel(args, dev, world, peaks, ranks=4, inputs=None):
     """Context-parallel (ring) attention on the 131K-token GQA workload split over ``ranks`` ranks,
     emulated on this GPU: each rank's steps (fused kernel + lse merge per visible key block) run
     back to back with the blocks already split; no exchange (its NVLink cost is not measured).
-    Reported beside one fused-kernel call over the whole sequence, both in bf16_exact."""
+    Reported beside one fused-kernel call over the whole sequence, both in bf16_exact.  Each step's
+    kernel runs ~14 ms, so the fraction is taken of the burst bf16 rate (the sustained one beside
+    it)."""
     import tiled_attention_22_b200 as ta
     from tiled_attention_22_b200.ring import ring_rank_emulated, ring_schedule
 
     w = WORKLOADS[5]
-    q, k, v = (t.to(dev) for t in make_inputs(w))
+    q, k, v = (t.to(dev) for t in (inputs if inputs is not None else make_inputs(w)))
     n = w.N // ranks
     qs = [q[:, :, r * n:(r + 1) * n].contiguous() for r in range(ranks)]
     kv = [(k[:, :, j * n:(j + 1) * n].contiguous(), v[:, :, j * n:(j + 1) * n].contiguous()) for j in range(ranks)]
@@ -551,11 +679,12 @@ def run_context_parallel(args, dev, world, peaks, ranks=4):
     steps = sum(kind != "skip" for r in range(ranks) for _, _, kind in ring_schedule(r, ranks, w.causal))
     tf = flops / (res["ring"] * 1e-3) / 1e12
     out = {w.name + f"_ring{ranks}": {
-        "ms_per_call": res["ring"], "TFLOP/s": tf * world, "frac_of_bf16_peak": tf / peaks["bf16_sustained"],
+        "ms_per_call": res["ring"], "TFLOP/s": tf * world, "frac_of_bf16_peak": tf / peaks["bf16"],
+        "frac_of_bf16_sustained": tf / peaks["bf16_sustained"],
         "single_call_ms": res["single_call"], "ring_over_single": res["ring"] / res["single_call"],
         "launches_per_call": 2 * steps, "kernels": "attn_fwd_persistent_kernel<128,bf16> + lse_merge_kernel<128,bf16>",
         "note": "all ranks' steps on one GPU; the key/value exchange over NVLink is not timed"}}
-    out["peak_note"] = "bf16 dense GEMM %.0f TFLOP/s (%s, sustained)" % (peaks["bf16_sustained"], peaks["source"])
+    out["peak_note"] = "bf16 dense GEMM %.0f TFLOP/s (%s, burst)" % (peaks["bf16"], peaks["source"])
     del q, k, v, qs, kv, o
     torch.cuda.empty_cache()
     return out
@@ -583,13 +712,15 @@ def _prepass_bytes(w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--config", type=int, default=5, help="headline workload (default: the 131072-token one)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the measurements of the other paths (KV-cache decode, prefix mask, ring)")
+    ap.add_argument("--no-others", action="store_true", help="skip the other workloads (N = 4096, 8192, 16384)")
+    ap.add_argument("--no-gemm-peaks", action="store_true", help="skip timing the 8-bit library GEMMs")
     ap.add_argument("--modes", default="int8_qk,bf16_exact,fp8_qk",
                     help="modes to time (the headline value is int8_qk; drop one only for profiling)")
     args = ap.parse_args()

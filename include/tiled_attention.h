@@ -27,8 +27,13 @@
  *     H = Hkv for K and V.  Query head h reads kv head h / (Hq / Hkv).
  *   - d must be 64 or 128.  N >= 1; N need not be a multiple of 128.
  *   - Every device pointer must be 16-byte aligned (TMA requirement).
- *   - All buffers belong to the caller.  The library allocates no memory and
- *     keeps no state beyond one device status word per GPU.
+ *   - All buffers belong to the caller.  The library allocates no memory.  Its
+ *     own state, per GPU, is fixed-size device data built into the library:
+ *     one device status word, 256 work-item counters of the persistent
+ *     attention kernel (attn_fwd) and the 8 MiB K-mean array of
+ *     attn_quant_smooth_k_noalloc.  The device addresses of the counters and
+ *     of that array are looked up on first use on each device and cached, so
+ *     the library must not be used across a cudaDeviceReset of that device.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and never synchronise, except attn_check_status and
  *     attn_fwd_host, which say so.
@@ -81,16 +86,19 @@ enum attn_dtype { ATTN_BF16 = 0, ATTN_FP16 = 1 };
  *     attn_workspace_bytes(B,Hq,Hkv,N,d,mode) bytes (0 for BF16_EXACT, where
  *     workspace may be NULL).  Its content on entry does not matter.
  *   Launches: BF16_EXACT with d = 128 runs on persistent CTAs (one per SM)
- *     that take 256-row work items from a counter inside the library, one
- *     counter per stream handle (256 per device; calls from further streams
- *     take one CTA per item, with the same results), cleared by a 4-byte
- *     cudaMemsetAsync on the stream before the kernel.  Calls on one stream are
- *     ordered by the stream and calls on different streams use different
- *     counters; a stream handle destroyed while its call still runs must not
- *     be reused by a new stream that calls this function before that call
- *     ends.  The first call on a device looks up the counters' address (with
- *     that device current): make it before any stream capture on the device.
- *     The other modes and d = 64 launch one CTA per work item.
+ *     that take 256-row work items from a counter inside the library, cleared
+ *     by a 4-byte cudaMemsetAsync on the stream before the kernel.  There is
+ *     one counter per stream, told apart by the stream's process-unique id
+ *     (cudaStreamGetId), so cudaStreamPerThread used from several host
+ *     threads, or a new stream that reuses a destroyed stream's handle value,
+ *     gets its own counter; calls on one stream are ordered by the stream.
+ *     A device has 256 counters; calls from further streams, and every call
+ *     made while its stream is being captured into a CUDA graph (a captured
+ *     counter address would be shared by every replay, on any stream), launch
+ *     one CTA per work item instead, with the same results.  The first call on
+ *     a device looks up the counters' address (with that device current):
+ *     make it before any stream capture on the device.  The other modes and
+ *     d = 64 launch one CTA per work item.
  */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int N, int d, int causal, float scale, int mode,
@@ -168,8 +176,9 @@ int attn_fwd_fp8_quantized(const uint8_t* q8, const float* sq, const uint8_t* k8
  *   N=131072, d=128); larger sizes return ATTN_ERR_WORKSPACE before launching (text in
  *   attn_last_cuda_error) and need attn_quant_smooth_k.
  *   The first call on each device looks up the array's device address (with that device
- *   current) and caches it; make that first call before any stream capture on that device.
- *   The call itself allocates nothing.  All calls on a device share the one array, and it keeps
+ *   current) and caches it; make that first call before any stream capture on that device, and
+ *   do not use the library across a cudaDeviceReset of that device (the cached address would
+ *   be stale).  The call itself allocates nothing.  All calls on a device share the one array, and it keeps
  *   the previous call's contents (every entry a call reads is written by the same call first):
  *   calls whose kernels overlap on the GPU (different streams, no ordering) race on it, so order
  *   them, for example by issuing them on one stream.

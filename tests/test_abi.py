@@ -148,3 +148,28 @@ def test_decode_workspace_sizes(lib):
     assert lib.attn_decode_workspace_bytes(1, 2, 2, 1, 256, 128, 50) == \
         lib.attn_decode_workspace_bytes(1, 2, 2, 1, 256, 128, 4)
     assert lib.attn_decode_workspace_bytes(1, 2, 2, 1, 256, 64, 2) == 0  # d = 64 unsupported
+
+
+class _FakeTensor:
+    """Stands in for a tensor in the binding's device check (only .device is read)."""
+
+    def __init__(self, kind, index=None):
+        import torch
+
+        self.device = torch.device(kind, index) if index is not None else torch.device(kind)
+
+
+def test_binding_refuses_tensors_on_two_devices():
+    """Every launch and the library's per-device state follow the current device, so a binding call
+    runs with its tensors' device current and refuses tensors spread over several devices."""
+    from tiled_attention_22_b200 import binding
+
+    a0, b0, a1 = _FakeTensor("cuda", 0), _FakeTensor("cuda", 0), _FakeTensor("cuda", 1)
+    assert binding._device_of(a0, None, b0) == 0
+    assert binding._device_of(None, a1) == 1
+    with pytest.raises(ValueError, match="one device"):
+        binding._device_of(a0, a1)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        binding._device_of(a0, _FakeTensor("cpu"))
+    with pytest.raises(ValueError, match="no CUDA tensor"):
+        binding._device_of(None, None)

@@ -3,8 +3,8 @@
   pre-pass: E4M3 codes (bit patterns), sq, sk, kmean bit-exact against O3; lse_bias within 1e-4.
   fused kernel: against O3 (the same codes; the GPU accumulates the exact code products in fp32)
     at the bf16_exact bars, and against exact attention O1 at the int8_qk bars (cosine >= 0.999,
-    scaled max error <= 5e-2, lse <= 5e-2) wherever O3 itself meets them, else within a small
-    margin of O3's own error.
+    max |o - O| - h|O| <= 5e-2 with h the output type's half-ulp, lse <= 5e-2) wherever O3 itself
+    meets them, else within a small margin of O3's own error (tests/tolerances.py).
 """
 import numpy as np
 import pytest
@@ -13,11 +13,9 @@ import torch
 import oracle
 from attn_workloads import WORKLOADS, Workload, make_inputs
 from oracle import fp8_emulation as f8
+from tolerances import INT8_COS as Q_COS, INT8_LSE as Q_LSE, INT8_MAX as Q_MAX, assert_close16, quant_metrics
 
 pytestmark = pytest.mark.gpu
-
-BF16_MAX, BF16_MEAN, BF16_LSE = 2e-2, 2e-3, 1e-3
-Q_COS, Q_MAX, Q_LSE = 0.999, 5e-2, 5e-2
 
 
 @pytest.fixture(scope="module")
@@ -36,26 +34,10 @@ def _np(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def scaled_err(o, O):
-    return np.abs(o - O) / np.maximum(1.0, np.abs(O))
-
-
-def cosine(a, b):
-    a, b = a.reshape(-1), b.reshape(-1)
-    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b) + 1e-300))
-
-
-def metrics(o, l, O, L):
-    return {"cos": cosine(o, O), "err": float(scaled_err(o, O).max()), "lse": float(np.abs(l - L).max())}
-
-
-def assert_fp8(o, l, O, L, Oe, Le, what):
+def assert_fp8(o, l, O, L, Oe, Le, what, dtype="bf16"):
     assert np.isfinite(o).all(), what
-    err = scaled_err(o, Oe)
-    assert err.max() <= BF16_MAX, f"{what}: vs emulation max err {err.max():.3e}"
-    assert err.mean() <= BF16_MEAN, f"{what}: vs emulation mean err {err.mean():.3e}"
-    assert np.abs(l - Le).max() <= BF16_LSE, f"{what}: vs emulation lse err {np.abs(l - Le).max():.3e}"
-    g, e = metrics(o, l, O, L), metrics(Oe, Le, O, L)
+    assert_close16(o, l, Oe, Le, dtype, f"{what}: vs emulation")
+    g, e = quant_metrics(o, l, O, L, dtype), quant_metrics(Oe, Le, O, L, dtype)
     if e["cos"] >= Q_COS and e["err"] <= Q_MAX and e["lse"] <= Q_LSE:
         assert g["cos"] >= Q_COS and g["err"] <= Q_MAX and g["lse"] <= Q_LSE, f"{what}: {g}"
     else:
@@ -118,7 +100,7 @@ def test_fp8_qk_small(ta, case):
     assert ta.attn_check_status() == 0
     O, L = oracle.attention(q, k, v, w.scale, causal)
     Oe, Le = emulated(q, k, v, causal, w.scale)
-    assert_fp8(_np(o), l.cpu().numpy().astype(np.float64), O, L, Oe, Le, str(case))
+    assert_fp8(_np(o), l.cpu().numpy().astype(np.float64), O, L, Oe, Le, str(case), dt)
 
 
 def test_fp8_fwd_equals_prepass_plus_fused(ta):

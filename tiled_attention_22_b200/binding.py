@@ -92,9 +92,33 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
+def _device_of(*tensors) -> int:
+    """The one CUDA device of a call's tensors (None entries are skipped).  The library resolves the
+    device of every launch, and of its per-device state, from the current device, so each call is
+    made with this device current; tensors on different devices are refused."""
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        d = t.device
+        if d.type != "cuda" or d.index is None:
+            raise ValueError("every device tensor of the call must be a CUDA tensor")
+        if dev is None:
+            dev = d.index
+        elif d.index != dev:
+            raise ValueError(f"tensors on cuda:{dev} and cuda:{d.index}: one call runs on one device")
+    if dev is None:
+        raise ValueError("the call has no CUDA tensor")
+    return dev
+
+
+def _stream(stream, dev=None):
+    """The cudaStream_t to pass: ``stream`` (a torch.cuda.Stream on the call's device), else the
+    current stream of that device."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
+    elif dev is not None and stream.device.index != dev:
+        raise ValueError(f"stream of cuda:{stream.device.index} for tensors on cuda:{dev}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -140,9 +164,12 @@ def attn_fwd(q, k, v, causal=False, scale=None, mode="bf16_exact", out=None, lse
     ws_bytes = attn_workspace_bytes(B, Hq, Hkv, N, d, mode)
     if ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
-    rc = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, int(bool(causal)), scale,
-                      MODES[mode], DTYPES[q.dtype], _ptr(workspace),
-                      0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
+    dev = _device_of(q, k, v, o, l, workspace)
+    with torch.cuda.device(dev):
+        rc = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, int(bool(causal)), scale,
+                          MODES[mode], DTYPES[q.dtype], _ptr(workspace),
+                          0 if workspace is None else workspace.numel() * workspace.element_size(),
+                          _stream(stream, dev))
     _check(rc, "attn_fwd")
     return o, l
 
@@ -176,8 +203,10 @@ def attn_fwd_prefix_masked(q, k, v, row_kv_limit, scale=None, out=None, lse=True
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty_like(q) if out is None else out
     l = _lse_arg(lse, (B, Hq, Nq), q.device)
-    rc = lib.attn_fwd_prefix_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, Nq, Nk, d,
-                                    _ptr(row_kv_limit), scale, DTYPES[q.dtype], _stream(stream))
+    dev = _device_of(q, k, v, o, l, row_kv_limit)
+    with torch.cuda.device(dev):
+        rc = lib.attn_fwd_prefix_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, Nq, Nk, d,
+                                        _ptr(row_kv_limit), scale, DTYPES[q.dtype], _stream(stream, dev))
     _check(rc, "attn_fwd_prefix_masked")
     return o, l
 
@@ -211,10 +240,12 @@ def attn_decode(q, k_cache, v_cache, kv_lens=None, causal=False, scale=None, num
     ws_bytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_ctas)
     if ws_bytes and workspace is None:  # (a reused workspace must have been zeroed once)
         workspace = torch.zeros(ws_bytes, device=q.device, dtype=torch.uint8)
-    rc = lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kv_lens), _ptr(o), _ptr(l), B, Hq, Hkv, Nq,
-                         Nk, d, int(bool(causal)), scale, DTYPES[q.dtype], int(num_ctas), _ptr(workspace),
-                         0 if workspace is None else workspace.numel() * workspace.element_size(),
-                         _stream(stream))
+    dev = _device_of(q, k_cache, v_cache, kv_lens, o, l, workspace)
+    with torch.cuda.device(dev):
+        rc = lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kv_lens), _ptr(o), _ptr(l), B, Hq, Hkv,
+                             Nq, Nk, d, int(bool(causal)), scale, DTYPES[q.dtype], int(num_ctas), _ptr(workspace),
+                             0 if workspace is None else workspace.numel() * workspace.element_size(),
+                             _stream(stream, dev))
     _check(rc, "attn_decode")
     return o, l
 
@@ -239,9 +270,11 @@ def attn_quant_smooth_k(q, k, scale=None, scratch=None, stream=None, out=None):
     nbytes = attn_quant_scratch_bytes(B, Hkv, N, d)
     if scratch is None:
         scratch = torch.empty(nbytes, device=dev, dtype=torch.uint8)
-    rc = lib.attn_quant_smooth_k(_ptr(q), _ptr(k), B, Hq, Hkv, N, d, DTYPES[q.dtype], scale, _ptr(out["q8"]),
-                                 _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]), _ptr(out["kmean"]),
-                                 _ptr(out["lse_bias"]), _ptr(scratch), scratch.numel(), _stream(stream))
+    dev = _device_of(q, k, scratch, *out.values())
+    with torch.cuda.device(dev):
+        rc = lib.attn_quant_smooth_k(_ptr(q), _ptr(k), B, Hq, Hkv, N, d, DTYPES[q.dtype], scale, _ptr(out["q8"]),
+                                     _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]), _ptr(out["kmean"]),
+                                     _ptr(out["lse_bias"]), _ptr(scratch), scratch.numel(), _stream(stream, dev))
     _check(rc, "attn_quant_smooth_k")
     return out
 
@@ -265,9 +298,11 @@ def attn_quant_smooth_k_noalloc(q, k, scale=None, out=None, stream=None):
         kmean=torch.empty((B, Hkv, d), device=dev, dtype=torch.float32),
         lse_bias=torch.empty((B, Hq, N), device=dev, dtype=torch.float32),
     )
-    rc = lib.attn_quant_smooth_k_noalloc(_ptr(q), _ptr(k), B, Hq, Hkv, N, d, DTYPES[q.dtype], scale,
-                                         _ptr(out["q8"]), _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]),
-                                         _ptr(out["kmean"]), _ptr(out["lse_bias"]), _stream(stream))
+    dev = _device_of(q, k, *out.values())
+    with torch.cuda.device(dev):
+        rc = lib.attn_quant_smooth_k_noalloc(_ptr(q), _ptr(k), B, Hq, Hkv, N, d, DTYPES[q.dtype], scale,
+                                             _ptr(out["q8"]), _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]),
+                                             _ptr(out["kmean"]), _ptr(out["lse_bias"]), _stream(stream, dev))
     _check(rc, "attn_quant_smooth_k_noalloc")
     return out
 
@@ -281,9 +316,11 @@ def attn_fwd_int8_quantized(pre, v, causal=False, scale=None, out=None, lse=True
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty((B, Hq, N, d), device=v.device, dtype=v.dtype) if out is None else out
     l = _lse_arg(lse, (B, Hq, N), v.device)
-    rc = lib.attn_fwd_int8_quantized(_ptr(q8), _ptr(pre["sq"]), _ptr(k8), _ptr(pre["sk"]), _ptr(pre["lse_bias"]),
-                                     _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, int(bool(causal)), scale,
-                                     DTYPES[v.dtype], _stream(stream))
+    dev = _device_of(q8, k8, pre["sq"], pre["sk"], pre["lse_bias"], v, o, l)
+    with torch.cuda.device(dev):
+        rc = lib.attn_fwd_int8_quantized(_ptr(q8), _ptr(pre["sq"]), _ptr(k8), _ptr(pre["sk"]),
+                                         _ptr(pre["lse_bias"]), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d,
+                                         int(bool(causal)), scale, DTYPES[v.dtype], _stream(stream, dev))
     _check(rc, "attn_fwd_int8_quantized")
     return o, l
 
@@ -308,9 +345,12 @@ def attn_quant_smooth_k_fp8(q, k, scale=None, scratch=None, stream=None, out=Non
     )
     if scratch is None:
         scratch = torch.empty(attn_quant_scratch_bytes(B, Hkv, N, d), device=dev, dtype=torch.uint8)
-    rc = lib.attn_quant_smooth_k_fp8(_ptr(q), _ptr(k), B, Hq, Hkv, N, d, DTYPES[q.dtype], scale, _ptr(out["q8"]),
-                                     _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]), _ptr(out["kmean"]),
-                                     _ptr(out["lse_bias"]), _ptr(scratch), scratch.numel(), _stream(stream))
+    dev = _device_of(q, k, scratch, *out.values())
+    with torch.cuda.device(dev):
+        rc = lib.attn_quant_smooth_k_fp8(_ptr(q), _ptr(k), B, Hq, Hkv, N, d, DTYPES[q.dtype], scale,
+                                         _ptr(out["q8"]), _ptr(out["sq"]), _ptr(out["k8"]), _ptr(out["sk"]),
+                                         _ptr(out["kmean"]), _ptr(out["lse_bias"]), _ptr(scratch), scratch.numel(),
+                                         _stream(stream, dev))
     _check(rc, "attn_quant_smooth_k_fp8")
     return out
 
@@ -324,9 +364,11 @@ def attn_fwd_fp8_quantized(pre, v, causal=False, scale=None, out=None, lse=True,
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty((B, Hq, N, d), device=v.device, dtype=v.dtype) if out is None else out
     l = _lse_arg(lse, (B, Hq, N), v.device)
-    rc = lib.attn_fwd_fp8_quantized(_ptr(q8), _ptr(pre["sq"]), _ptr(k8), _ptr(pre["sk"]), _ptr(pre["lse_bias"]),
-                                    _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, int(bool(causal)), scale,
-                                    DTYPES[v.dtype], _stream(stream))
+    dev = _device_of(q8, k8, pre["sq"], pre["sk"], pre["lse_bias"], v, o, l)
+    with torch.cuda.device(dev):
+        rc = lib.attn_fwd_fp8_quantized(_ptr(q8), _ptr(pre["sq"]), _ptr(k8), _ptr(pre["sk"]),
+                                        _ptr(pre["lse_bias"]), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d,
+                                        int(bool(causal)), scale, DTYPES[v.dtype], _stream(stream, dev))
     _check(rc, "attn_fwd_fp8_quantized")
     return o, l
 
@@ -338,8 +380,10 @@ def attn_probe_qk_int32(q8, k8, tiles, stream=None):
     Hkv = k8.shape[1]
     t = torch.tensor(tiles, dtype=torch.int32).reshape(-1, 4).to(q8.device)
     out = torch.empty((t.shape[0], 128, 128), device=q8.device, dtype=torch.int32)
-    rc = lib.attn_probe_qk_int32(_ptr(q8), _ptr(k8), B, Hq, Hkv, N, d, _ptr(t), t.shape[0], _ptr(out),
-                                 _stream(stream))
+    dev = _device_of(q8, k8, t, out)
+    with torch.cuda.device(dev):
+        rc = lib.attn_probe_qk_int32(_ptr(q8), _ptr(k8), B, Hq, Hkv, N, d, _ptr(t), t.shape[0], _ptr(out),
+                                     _stream(stream, dev))
     _check(rc, "attn_probe_qk_int32")
     return out
 
@@ -351,10 +395,12 @@ def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, dq, dk, dv, do_, dls
     B, Hq, N, d = q_host.shape
     Hkv = k_host.shape[1]
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib.attn_fwd_host(_ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host), _ptr(lse_host), _ptr(dq),
-                           _ptr(dk), _ptr(dv), _ptr(do_), _ptr(dlse), B, Hq, Hkv, N, d, int(bool(causal)), scale,
-                           MODES[mode], DTYPES[q_host.dtype], _ptr(workspace),
-                           0 if workspace is None else workspace.numel(), _stream(stream))
+    dev = _device_of(dq, dk, dv, do_, dlse, workspace)
+    with torch.cuda.device(dev):
+        rc = lib.attn_fwd_host(_ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host), _ptr(lse_host), _ptr(dq),
+                               _ptr(dk), _ptr(dv), _ptr(do_), _ptr(dlse), B, Hq, Hkv, N, d, int(bool(causal)),
+                               scale, MODES[mode], DTYPES[q_host.dtype], _ptr(workspace),
+                               0 if workspace is None else workspace.numel(), _stream(stream, dev))
     _check(rc, "attn_fwd_host")
 
 
@@ -381,8 +427,10 @@ def attn_merge_lse(o_acc, lse_acc, o_part=None, lse_part=None, out=None, first=F
             raise ValueError("o_part and out must be 16-bit tensors of o_acc's size and one dtype")
     if lse_part is not None and (lse_part.dtype != torch.float32 or lse_part.numel() != rows):
         raise ValueError("lse_part must be float32 with one value per row")
-    rc = lib.attn_merge_lse(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part), _ptr(out), rows, d,
-                            DTYPES[ref.dtype], int(bool(first)), _stream(stream))
+    dev = _device_of(o_acc, lse_acc, o_part, lse_part, out)
+    with torch.cuda.device(dev):
+        rc = lib.attn_merge_lse(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part), _ptr(out), rows, d,
+                                DTYPES[ref.dtype], int(bool(first)), _stream(stream, dev))
     _check(rc, "attn_merge_lse")
     return out
 
@@ -404,6 +452,8 @@ def attn_test_exp2(x, use_poly, stream=None):
     """Apply the kernel's exp2 routine to a float32 CUDA tensor: use_poly 0 = MUFU ex2.approx,
     1 = FMA-pipe polynomial, 2 = the polynomial on packed pairs."""
     y = torch.empty_like(x)
-    _check(load_library().attn_test_exp2(_ptr(x), _ptr(y), x.numel(), int(use_poly), _stream(stream)),
-           "attn_test_exp2")
+    dev = _device_of(x, y)
+    with torch.cuda.device(dev):
+        _check(load_library().attn_test_exp2(_ptr(x), _ptr(y), x.numel(), int(use_poly), _stream(stream, dev)),
+               "attn_test_exp2")
     return y

@@ -7,18 +7,35 @@
 #define TATTN_SPLIT 0
 #endif
 
-// Persistent launches take their work items from a ticket counter, one per (device, stream) so that
-// launches on different streams never share one; it is cleared on the stream before each launch.
-// The counters live in the library, kTicketSlots per device; launches from further streams use one
-// CTA per item instead (the same results).
+// Persistent launches take their work items from a ticket counter that no other launch may touch
+// while they run; the counter is cleared on the launch's stream just before the kernel.  Counters
+// live in the library, kTicketSlots per device, one per stream, keyed by the stream's id
+// (cudaStreamGetId: unique in the process for the life of the program).  The id, unlike the handle
+// value, tells apart streams that share a handle: cudaStreamPerThread names a different stream in
+// each host thread, and a destroyed stream's handle value can come back for a new stream.  Launches
+// from streams past the kTicketSlots-th use one CTA per item instead (the same results).
+//
+// A launch recorded by stream capture would carry its counter's address into every replay of the
+// graph, on whatever stream the replay runs, alongside direct calls on the capturing stream; so a
+// capturing stream gets no counter and the launch uses one CTA per item.
 constexpr int kTicketSlots = 256;
 __device__ unsigned g_fwd_tickets[kTicketSlots];
 
 unsigned* fwd_ticket_counter(cudaStream_t stream) {
   static std::mutex mu;
   static unsigned* base[kMaxDevices];
-  static cudaStream_t owner[kMaxDevices][kTicketSlots];
+  static unsigned long long owner[kMaxDevices][kTicketSlots];
   static int used[kMaxDevices];
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess || capture != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  unsigned long long id = 0;
+  if (cudaStreamGetId(stream, &id) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
@@ -34,9 +51,9 @@ unsigned* fwd_ticket_counter(cudaStream_t stream) {
     base[dev] = static_cast<unsigned*>(addr);
   }
   for (int i = 0; i < used[dev]; ++i)
-    if (owner[dev][i] == stream) return base[dev] + i;
+    if (owner[dev][i] == id) return base[dev] + i;
   if (used[dev] == kTicketSlots) return nullptr;
-  owner[dev][used[dev]] = stream;
+  owner[dev][used[dev]] = id;
   return base[dev] + used[dev]++;
 }
 
