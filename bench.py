@@ -474,7 +474,7 @@ def run_native(args, w, world, rank, local):
         torch.cuda.synchronize()
         ems, e2e_tflops = whole_job_rate(s0.elapsed_time(s1), w.flops() * e_steps, world)
         e2e = {"value": e2e_tflops, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": int(3 * q.numel() * q.element_size()),
+               "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * q.element_size()),
                "d2h_bytes_per_step": int(o.numel() * o.element_size() + lse.numel() * 4),
                "steps": e_steps, "ms_per_step": ems / e_steps}
         del qh, kh, vh, oh, lh, ws

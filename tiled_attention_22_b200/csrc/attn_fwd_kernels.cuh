@@ -39,11 +39,18 @@
 
 namespace tattn {
 
+// Query rows per work item: two 128-row tiles that ping-pong on the tensor cores (the default), or
+// one tile (TATTN_QT1: a measurement variant showing what the second tile buys).
+#ifndef TATTN_QT1
+#define TATTN_QT1 0
+#endif
+constexpr int kItemRows = TATTN_QT1 ? 128 : 256;
+
 struct FwdParams {
   int B, Hq, Hkv, N, causal;  // N: query rows
   int Nk;                 // keys (= N except under a row prefix mask)
   const int* row_lim;     // [N] or null: query row i sees keys j < row_lim[i] (clamped to [0, Nk])
-  int n_mblocks;          // ceil(N / 256)
+  int n_mblocks;          // ceil(N / kItemRows)
   int sec_kv;             // kv heads per scheduling section (K/V of a section stay in L2)
   float scale_log2;       // scale * log2(e)
   void* o;                // [B, Hq, N, D] 16-bit
@@ -77,10 +84,13 @@ struct FwdCfg {
 #ifndef TATTN_POLY_D128
 #define TATTN_POLY_D128 0
 #endif
+#ifndef TATTN_POLY_D128_BYTE
+#define TATTN_POLY_D128_BYTE TATTN_POLY_D128
+#endif
 #ifndef TATTN_POLY_D64
 #define TATTN_POLY_D64 4
 #endif
-  static constexpr int POLY_PER_16 = D == 64 ? TATTN_POLY_D64 : TATTN_POLY_D128;
+  static constexpr int POLY_PER_16 = D == 64 ? TATTN_POLY_D64 : (BYTE ? TATTN_POLY_D128_BYTE : TATTN_POLY_D128);
   // pipeline depth (K and V rings); defaults chosen by measurement on the named workloads
 #ifndef TATTN_KS_128B
 #define TATTN_KS_128B 2
@@ -128,8 +138,8 @@ struct FwdCfg {
   static constexpr int OFF_O = OFF_V + VSTAGES * V_TILE;
   static constexpr int OFF_BAR = OFF_O + O_STAGE;
   // barriers: q_full[2] k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2] o_done[2]
-  // drain, then (P in shared memory) s_free[2] pv_done[2]
-  static constexpr int NBAR = 2 + 2 * KSTAGES + 2 * VSTAGES + 6 + 1 + 4;
+  // drain, then (P in shared memory) s_free[2] pv_done[2], then p_half[2]
+  static constexpr int NBAR = 2 + 2 * KSTAGES + 2 * VSTAGES + 6 + 1 + 4 + 2;
   static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 32;  // + TMEM slot, abort flag, row-limit stats
   // +1024 for manual alignment of the dynamic shared memory base; at least 120 KB so that exactly
   // one CTA (which owns all 512 TMEM columns) is resident per SM.
@@ -142,6 +152,14 @@ struct FwdCfg {
 
 #ifndef TATTN_PFULL_PER_WARP
 #define TATTN_PFULL_PER_WARP 1
+#endif
+// P released in two halves: the softmax warps arrive on p_half once the first 64 columns of P are
+// in tensor memory and on p_full once all 128 are, so the first half of P V (keys 0..63 of the
+// tile) runs on the tensor cores while the softmax still computes the second half.  That takes
+// half a P V off each tile's Q K^T -> softmax -> P V chain.  Used with one thread per score row and
+// P in tensor memory (the default variants).
+#ifndef TATTN_PSPLIT
+#define TATTN_PSPLIT 1
 #endif
 
 // Warp roles.  Softmax warps come first, then one producer warpgroup (TMA warp, MMA warp, 2 idle).
@@ -201,12 +219,13 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint3
   }
 }
 
-// Issue O(tmem) (+)= P(tmem, 16-bit, K-major) * V_tile(smem, MN-major, 128B swizzle).
-template <int D, bool FP16>
+// Issue O(tmem) (+)= P(tmem, 16-bit, K-major) * V_tile(smem, MN-major, 128B swizzle), over keys
+// [16 K0, 16 K1) of the tile (all 128 by default).
+template <int D, bool FP16, int K0 = 0, int K1 = 128 / 16>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
   constexpr uint32_t idesc = instr_desc(1, FP16 ? 0 : 1, 0, 1, 128, D);
 #pragma unroll
-  for (int kk = 0; kk < 128 / 16; ++kk) {
+  for (int kk = K0; kk < K1; ++kk) {
     // 16 keys per step = 16 rows of 128 B; 64-column panels of V are 128 x 128 B apart (LBO),
     // groups of 8 key rows are 1024 B apart (SBO).
     const uint64_t bd = smem_desc(v_smem + kk * 16 * 128, 128 * 128, 1024, kSwizzle128B);
@@ -286,9 +305,10 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
-template <int D, int QK, bool FP16, bool MASKED>
+template <int D, int QK, bool FP16, bool MASKED, bool PS = false>
 __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc, int lim, int j, float& m_run,
-                                             float& l_run, uint64_t* o_done_t, volatile int* abort_flag) {
+                                             float& l_run, uint64_t* o_done_t, volatile int* abort_flag,
+                                             uint64_t* p_half_t = nullptr) {
   constexpr bool INT8 = QK == QK_I8;  // int32 scores (the FP8 kind's are fp32 like the 16-bit one's)
   using C = FwdCfg<D, QK != QK_F16>;
   uint32_t r[4][32];
@@ -334,8 +354,31 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
   const float2 sc2 = make_float2(sc, sc), cst2 = make_float2(-m_use, -m_use);
   const float2 off2 = make_float2(-12582912.0f, -12582912.0f);
   float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
+  if (PS && rescale && j > 0) {
+    // (P released in halves) O is rescaled before any of P(j) is released: the first half of
+    // P V(j) may start as soon as p_half completes.  O holds the P V sums of key tiles 0..j-1, and
+    // P V(j-1) has completed: the s_full commit that woke this thread was made after S(j), i.e.
+    // after P V(j-1) was issued by the same thread, and a commit tracks every earlier tcgen05
+    // operation of its thread.
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + 32 * c, o);
+      tmem_ld_wait(o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+      tmem_st32(tO + 32 * c, o);
+    }
+  }
 #pragma unroll
   for (int qtr = 0; qtr < 4; ++qtr) {
+    if (PS && qtr == 2) {
+      // the first 64 columns of P (and any O rescale) are in tensor memory: release them
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(p_half_t);
+    }
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -361,7 +404,7 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
     tmem_st16(tS + 16 * qtr, pk);
   }
   l_run += (ls0.x + ls0.y) + (ls1.x + ls1.y);
-  if (rescale && j > 0) {
+  if (!PS && rescale && j > 0) {
     // O holds the P V sums of key tiles 0..j-1.  The s_full commit that woke this thread was made
     // after S(j), i.e. after P V(j-1) was issued by the same thread, and a commit tracks every
     // earlier tcgen05 operation of its thread: P V(j-1) has completed.  P V(j) is issued only
@@ -611,7 +654,10 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
   uint64_t* drain = o_done + 2;
   uint64_t* s_free = drain + 1;    // P in shared memory only
   uint64_t* pv_done = s_free + 2;  // P in shared memory only
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
+  uint64_t* p_half = pv_done + 2;  // P released in halves only
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(p_half + 2);
+  // P released in halves: one thread per score row with P in tensor memory
+  constexpr bool PS = TATTN_PSPLIT && !SPLIT && !C::PSMEM;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -624,6 +670,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       mbar_init(&o_done[i], 1);
       mbar_init(&s_free[i], R::kThreadsPerTile / 32);
       mbar_init(&pv_done[i], 1);
+      mbar_init(&p_half[i], R::kThreadsPerTile / 32);
     }
     for (int i = 0; i < C::KSTAGES; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < C::VSTAGES; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
@@ -677,7 +724,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         int mx = 0, mn = INT_MAX;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int row = mb * 256 + 128 * t + 32 * k + lane;
+          const int row = mb * kItemRows + 128 * t + 32 * k + lane;
           if (row < p.N) {
             const int l = min(max(__ldg(&p.row_lim[row]), 0), p.Nk);
             mx = max(mx, l);
@@ -696,8 +743,8 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
   }
   // key tiles each query tile visits (0 for a tile past N); n1 >= n0 unless tile 1 is empty
   auto key_tiles = [&](int t) {
-    const int row0 = mb * 256 + 128 * t;
-    if (row0 >= p.N) return 0;
+    const int row0 = mb * kItemRows + 128 * t;
+    if (row0 >= p.N || (TATTN_QT1 && t == 1)) return 0;
     if (p.row_lim != nullptr) return (lim_stats[2 * t] + 127) / 128;
     return p.causal ? min(nkv, row0 / 128 + 1) : nkv;
   };
@@ -723,7 +770,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         if (n_of(t) == 0) continue;
         mbar_arrive_expect_tx(&q_full[t], C::Q_TILE);
         for (int pn = 0; pn < C::QK_PANELS; ++pn)
-          tma_load_3d(sQ + t * C::Q_TILE + pn * C::QK_PANEL_BYTES, &tmQ, pn * C::QK_BOX_X, mb * 256 + 128 * t, bh,
+          tma_load_3d(sQ + t * C::Q_TILE + pn * C::QK_PANEL_BYTES, &tmQ, pn * C::QK_BOX_X, mb * kItemRows + 128 * t, bh,
                       &q_full[t], pol_stream);
       }
       for (int j = 0; j < nmax && ok; ++j) {
@@ -843,13 +890,21 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         const int ks1 = (j + 1) % C::KSTAGES;
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= n_of(t)) continue;
-          if (!(ok = mbar_wait(&p_full[t], j & 1, abort_flag, W_MMA + 3))) break;
+          if (!(ok = mbar_wait(PS ? &p_half[t] : &p_full[t], j & 1, abort_flag, W_MMA + 3))) break;
           tc_fence_after();
           if (users_first(j) == t) {
             if (!(ok = mbar_wait(&v_full[vs], (j / C::VSTAGES) & 1, abort_flag, W_MMA + 4))) break;
             tc_fence_after();
           }
-          issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
+          if constexpr (PS) {
+            // keys 0..63 of the tile as soon as their P is in, the rest once all of P is
+            issue_pv<D, FP16, 0, 4>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
+            if (!(ok = mbar_wait(&p_full[t], j & 1, abort_flag, W_MMA + 6))) break;
+            tc_fence_after();
+            issue_pv<D, FP16, 4, 8>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, true);
+          } else {
+            issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
+          }
           if (j + 1 == n_of(t)) mma_commit(&o_done[t]);  // the tile's last P V: O is final
           if (users_last(j) == t) mma_commit(&v_empty[vs]);
           if (j + 1 < n_of(t)) {
@@ -880,7 +935,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       const int half = (warp >> 2) & 1;         // which 16 lanes of the quarter
       const int lane_base = wq * 32 + half * 16;
       const int nt = n_of(t);
-      const int row0 = mb * 256 + 128 * t;
+      const int row0 = mb * kItemRows + 128 * t;
       const int rowA = row0 + lane_base + (lane >> 2), rowB = rowA + 8;
       const uint32_t tS = tmem + C::tm_s(t) + ((uint32_t)lane_base << 16);
       const uint32_t tO = tmem + C::tm_o(t) + ((uint32_t)lane_base << 16);
@@ -970,7 +1025,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       // ================================ softmax (one row per thread) ================================
       const int t = warp >> 2, wq = warp & 3;
       const int nt = n_of(t);
-      const int row0 = mb * 256 + 128 * t;
+      const int row0 = mb * kItemRows + 128 * t;
       const int row = row0 + wq * 32 + lane;
       const uint32_t tS = tmem + C::tm_s(t) + ((uint32_t)(wq * 32) << 16);
       const uint32_t tO = tmem + C::tm_o(t) + ((uint32_t)(wq * 32) << 16);
@@ -1028,9 +1083,11 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         } else {
           if (diag || (col0 + 128 > p.Nk) || (col0 + 128 > tile_min_lim)) {
             const int lim = (p.row_lim != nullptr ? row_lim : (diag ? min(row + 1, p.Nk) : p.Nk)) - col0;
-            ok = softmax_step<D, QK, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
+            ok = softmax_step<D, QK, FP16, true, PS>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag,
+                                                     &p_half[t]);
           } else {
-            ok = softmax_step<D, QK, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
+            ok = softmax_step<D, QK, FP16, false, PS>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag,
+                                                      &p_half[t]);
           }
           if (!ok) break;
         }
@@ -1045,7 +1102,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
           mbar_arrive(&p_full[t]);
         }
       }
-      if (ok && nt == 0 && p.row_lim != nullptr && row < p.N) {
+      if (ok && nt == 0 && p.row_lim != nullptr && row < p.N && !(TATTN_QT1 && t == 1)) {
         // every row of this tile sees no key: O = 0, lse = -inf
         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.o) + ((size_t)bh * p.N + row) * (D * 2));
 #pragma unroll

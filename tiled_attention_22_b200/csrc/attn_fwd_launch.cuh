@@ -102,7 +102,10 @@ int launch_fwd_t(const void* q, const void* k, const void* v, const FwdParams& p
   // Persistent CTAs (one per SM) for 16-bit Q K^T at d = 128, where they measured 3-6% faster on
   // the named workloads (the 8-bit modes and d = 64 measured no gain); not under a row prefix mask
   // (its per-tile limits are read once per CTA) nor with the four-threads-per-row variant.
-  if constexpr (QK == QK_F16 && D == 128 && !SPLIT) {
+#ifndef TATTN_PERSIST_BYTE
+#define TATTN_PERSIST_BYTE 0
+#endif
+  if constexpr ((QK == QK_F16 || TATTN_PERSIST_BYTE) && D == 128 && !SPLIT) {
     unsigned* tickets = p.row_lim == nullptr && items <= 0x7fffffffll ? fwd_ticket_counter(stream) : nullptr;
     if (tickets != nullptr) {
       using PC = FwdPersistCfg<D, BYTE>;
@@ -144,7 +147,7 @@ FwdParams make_params(int B, int Hq, int Hkv, int N, int causal, float scale, vo
   p.Nk = Nk < 0 ? N : Nk;
   p.row_lim = row_lim;
   p.causal = causal;
-  p.n_mblocks = (N + 255) / 256;
+  p.n_mblocks = (N + kItemRows - 1) / kItemRows;
   // Scheduling sections: kv heads whose K and V (16-bit, d=128, the larger case) take at most
   // TATTN_L2_SECTION_MB (a quarter of the 126 MB L2 by default).
 #ifndef TATTN_L2_SECTION_MB

@@ -22,6 +22,12 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_
     std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
     return ATTN_ERR_LAUNCH;
   }
+  // The encoder is a driver call and needs the device's context current on this thread.  A host
+  // thread that has made no runtime call needing a context yet (a new thread whose streams came
+  // from a pool) has none; cudaSetDevice on the current device makes its primary context current.
+  int dev = 0;
+  TATTN_CUDA(cudaGetDevice(&dev));
+  TATTN_CUDA(cudaSetDevice(dev));
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * elem_bytes, (cuuint64_t)N * d * elem_bytes};
   cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1u};
