@@ -138,8 +138,8 @@ struct FwdCfg {
   static constexpr int OFF_O = OFF_V + VSTAGES * V_TILE;
   static constexpr int OFF_BAR = OFF_O + O_STAGE;
   // barriers: q_full[2] k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2] o_done[2]
-  // drain, then (P in shared memory) s_free[2] pv_done[2], then p_half[2]
-  static constexpr int NBAR = 2 + 2 * KSTAGES + 2 * VSTAGES + 6 + 1 + 4 + 2;
+  // drain, then (P in shared memory) s_free[2] pv_done[2]
+  static constexpr int NBAR = 2 + 2 * KSTAGES + 2 * VSTAGES + 6 + 1 + 4;
   static constexpr int SMEM_USED = OFF_BAR + NBAR * 8 + 32;  // + TMEM slot, abort flag, row-limit stats
   // +1024 for manual alignment of the dynamic shared memory base; at least 120 KB so that exactly
   // one CTA (which owns all 512 TMEM columns) is resident per SM.
@@ -153,14 +153,7 @@ struct FwdCfg {
 #ifndef TATTN_PFULL_PER_WARP
 #define TATTN_PFULL_PER_WARP 1
 #endif
-// P released in two halves: the softmax warps arrive on p_half once the first 64 columns of P are
-// in tensor memory and on p_full once all 128 are, so the first half of P V (keys 0..63 of the
-// tile) runs on the tensor cores while the softmax still computes the second half.  That takes
-// half a P V off each tile's Q K^T -> softmax -> P V chain.  Used with one thread per score row and
-// P in tensor memory (the default variants).
-#ifndef TATTN_PSPLIT
-#define TATTN_PSPLIT 1
-#endif
+
 
 // Warp roles.  Softmax warps come first, then one producer warpgroup (TMA warp, MMA warp, 2 idle).
 //   SPLIT = false: 8 softmax warps, one thread per score row (32x32b TMEM accesses).
@@ -219,13 +212,12 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint3
   }
 }
 
-// Issue O(tmem) (+)= P(tmem, 16-bit, K-major) * V_tile(smem, MN-major, 128B swizzle), over keys
-// [16 K0, 16 K1) of the tile (all 128 by default).
-template <int D, bool FP16, int K0 = 0, int K1 = 128 / 16>
+// Issue O(tmem) (+)= P(tmem, 16-bit, K-major) * V_tile(smem, MN-major, 128B swizzle).
+template <int D, bool FP16>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
   constexpr uint32_t idesc = instr_desc(1, FP16 ? 0 : 1, 0, 1, 128, D);
 #pragma unroll
-  for (int kk = K0; kk < K1; ++kk) {
+  for (int kk = 0; kk < 128 / 16; ++kk) {
     // 16 keys per step = 16 rows of 128 B; 64-column panels of V are 128 x 128 B apart (LBO),
     // groups of 8 key rows are 1024 B apart (SBO).
     const uint64_t bd = smem_desc(v_smem + kk * 16 * 128, 128 * 128, 1024, kSwizzle128B);
@@ -305,25 +297,8 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
-template <int D, int QK, bool FP16, bool MASKED, bool PS = false>
-__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc, int lim, int j, float& m_run,
-                                             float& l_run, uint64_t* o_done_t, volatile int* abort_flag,
-                                             uint64_t* p_half_t = nullptr) {
-  constexpr bool INT8 = QK == QK_I8;  // int32 scores (the FP8 kind's are fp32 like the 16-bit one's)
-  using C = FwdCfg<D, QK != QK_F16>;
-  uint32_t r[4][32];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
-  float x[128];
-#pragma unroll
-  for (int i = 0; i < 128; ++i) {
-    const uint32_t bits = r[i >> 5][i & 31];
-    // INT8: exact int32 -> float for |acc| < 2^22 (here |acc| <= 128 * 127^2): x = 1.5*2^23 + acc
-    x[i] = INT8 ? __uint_as_float(bits + 0x4B400000u) : __uint_as_float(bits);
-    if (MASKED && i >= lim) x[i] = -INFINITY;
-  }
+// Row maximum of the tile's scores (raw: x, or 1.5*2^23 + acc for INT8 scores).
+__device__ __forceinline__ float row_max128(const float (&x)[128]) {
   float mc[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -332,8 +307,61 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
     for (int k = 1; k < 31; k += 2) m = max3f(m, x[32 * c + k], x[32 * c + k + 1]);
     mc[c] = fmaxf(m, x[32 * c + 31]);
   }
-  const float mx = max3f(mc[0], mc[1], fmaxf(mc[2], mc[3]));
-  const float m_tile = INT8 ? (mx - 12582912.0f) * sc : mx * sc;
+  return max3f(mc[0], mc[1], fmaxf(mc[2], mc[3]));
+}
+
+// Row maximum of a tile of int32 scores (eight chains of two-input maxima).
+__device__ __forceinline__ int row_max128_i32(const uint32_t (&r)[4][32]) {
+  int mc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    int m = max((int)r[c >> 1][(c & 1) * 16], (int)r[c >> 1][(c & 1) * 16 + 1]);
+#pragma unroll
+    for (int k = 2; k < 16; ++k) m = max(m, (int)r[c >> 1][(c & 1) * 16 + k]);
+    mc[c] = m;
+  }
+  return max(max(max(mc[0], mc[1]), max(mc[2], mc[3])), max(max(mc[4], mc[5]), max(mc[6], mc[7])));
+}
+
+// INT8 scores, unmasked tiles, d = 128: the row maximum is taken on the int32 scores as loaded, and
+// their conversion to float (one integer add each) is left to the exponential loop, where it
+// overlaps the MUFU work instead of preceding the maximum.  Measured +2-4% on the 8192- and
+// 131072-token workloads; at d = 64 (where the exponentials outweigh the MMA work twice over) it
+// measured -2%, so d = 64 converts first.
+#ifndef TATTN_I8_LATE
+#define TATTN_I8_LATE 1
+#endif
+
+template <int D, int QK, bool FP16, bool MASKED>
+__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc, int lim, int j, float& m_run,
+                                             float& l_run, uint64_t* o_done_t, volatile int* abort_flag) {
+  constexpr bool INT8 = QK == QK_I8;  // int32 scores (the FP8 kind's are fp32 like the 16-bit one's)
+  using C = FwdCfg<D, QK != QK_F16>;
+  uint32_t r[4][32];
+  float x[128];
+  // INT8: exact int32 -> float for |acc| < 2^22 (here |acc| <= 128 * 127^2): x = 1.5*2^23 + acc
+  auto to_x = [&](int c) {
+#pragma unroll
+    for (int i = 32 * c; i < 32 * c + 32; ++i) {
+      const uint32_t bits = r[i >> 5][i & 31];
+      x[i] = INT8 ? __uint_as_float(bits + 0x4B400000u) : __uint_as_float(bits);
+      if (MASKED && i >= lim) x[i] = -INFINITY;
+    }
+  };
+  constexpr bool LATE = INT8 && !MASKED && D == 128 && TATTN_I8_LATE;
+  float m_tile;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, r[c]);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld_wait(r[c]);
+  if (LATE) {
+    m_tile = (float)row_max128_i32(r) * sc;  // |acc| < 2^22: exact
+  } else {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) to_x(c);
+    const float mx = row_max128(x);
+    m_tile = INT8 ? (mx - 12582912.0f) * sc : mx * sc;
+  }
   // Each row decides for itself whether its running max moves (so its rounding never depends on
   // other rows); the TMEM rescale of O below is warp-uniform (.aligned), and rows that keep their
   // max multiply by exactly 1.
@@ -354,31 +382,12 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
   const float2 sc2 = make_float2(sc, sc), cst2 = make_float2(-m_use, -m_use);
   const float2 off2 = make_float2(-12582912.0f, -12582912.0f);
   float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
-  if (PS && rescale && j > 0) {
-    // (P released in halves) O is rescaled before any of P(j) is released: the first half of
-    // P V(j) may start as soon as p_half completes.  O holds the P V sums of key tiles 0..j-1, and
-    // P V(j-1) has completed: the s_full commit that woke this thread was made after S(j), i.e.
-    // after P V(j-1) was issued by the same thread, and a commit tracks every earlier tcgen05
-    // operation of its thread.
+  if (LATE) {
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t o[32];
-      tmem_ld32(tO + 32 * c, o);
-      tmem_ld_wait(o);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-      tmem_st32(tO + 32 * c, o);
-    }
+    for (int c = 0; c < 4; ++c) to_x(c);
   }
 #pragma unroll
   for (int qtr = 0; qtr < 4; ++qtr) {
-    if (PS && qtr == 2) {
-      // the first 64 columns of P (and any O rescale) are in tensor memory: release them
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if ((threadIdx.x & 31) == 0) mbar_arrive(p_half_t);
-    }
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -404,7 +413,7 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, float sc,
     tmem_st16(tS + 16 * qtr, pk);
   }
   l_run += (ls0.x + ls0.y) + (ls1.x + ls1.y);
-  if (!PS && rescale && j > 0) {
+  if (rescale && j > 0) {
     // O holds the P V sums of key tiles 0..j-1.  The s_full commit that woke this thread was made
     // after S(j), i.e. after P V(j-1) was issued by the same thread, and a commit tracks every
     // earlier tcgen05 operation of its thread: P V(j-1) has completed.  P V(j) is issued only
@@ -654,10 +663,7 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
   uint64_t* drain = o_done + 2;
   uint64_t* s_free = drain + 1;    // P in shared memory only
   uint64_t* pv_done = s_free + 2;  // P in shared memory only
-  uint64_t* p_half = pv_done + 2;  // P released in halves only
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(p_half + 2);
-  // P released in halves: one thread per score row with P in tensor memory
-  constexpr bool PS = TATTN_PSPLIT && !SPLIT && !C::PSMEM;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -670,7 +676,6 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
       mbar_init(&o_done[i], 1);
       mbar_init(&s_free[i], R::kThreadsPerTile / 32);
       mbar_init(&pv_done[i], 1);
-      mbar_init(&p_half[i], R::kThreadsPerTile / 32);
     }
     for (int i = 0; i < C::KSTAGES; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < C::VSTAGES; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
@@ -890,21 +895,13 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         const int ks1 = (j + 1) % C::KSTAGES;
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= n_of(t)) continue;
-          if (!(ok = mbar_wait(PS ? &p_half[t] : &p_full[t], j & 1, abort_flag, W_MMA + 3))) break;
+          if (!(ok = mbar_wait(&p_full[t], j & 1, abort_flag, W_MMA + 3))) break;
           tc_fence_after();
           if (users_first(j) == t) {
             if (!(ok = mbar_wait(&v_full[vs], (j / C::VSTAGES) & 1, abort_flag, W_MMA + 4))) break;
             tc_fence_after();
           }
-          if constexpr (PS) {
-            // keys 0..63 of the tile as soon as their P is in, the rest once all of P is
-            issue_pv<D, FP16, 0, 4>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
-            if (!(ok = mbar_wait(&p_full[t], j & 1, abort_flag, W_MMA + 6))) break;
-            tc_fence_after();
-            issue_pv<D, FP16, 4, 8>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, true);
-          } else {
-            issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
-          }
+          issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
           if (j + 1 == n_of(t)) mma_commit(&o_done[t]);  // the tile's last P V: O is final
           if (users_last(j) == t) mma_commit(&v_empty[vs]);
           if (j + 1 < n_of(t)) {
@@ -1083,11 +1080,9 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         } else {
           if (diag || (col0 + 128 > p.Nk) || (col0 + 128 > tile_min_lim)) {
             const int lim = (p.row_lim != nullptr ? row_lim : (diag ? min(row + 1, p.Nk) : p.Nk)) - col0;
-            ok = softmax_step<D, QK, FP16, true, PS>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag,
-                                                     &p_half[t]);
+            ok = softmax_step<D, QK, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
           } else {
-            ok = softmax_step<D, QK, FP16, false, PS>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag,
-                                                      &p_half[t]);
+            ok = softmax_step<D, QK, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
           }
           if (!ok) break;
         }

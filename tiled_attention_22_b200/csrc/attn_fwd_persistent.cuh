@@ -20,7 +20,7 @@ enum : int { W_ITEM = 0x70 };
 
 // Shared-memory layout: attn_fwd_kernel's tiles and O staging, then the barriers
 //   q_full[2] q_empty[2] k_full[KS] k_empty[KS] v_full[VS] v_empty[VS] s_full[2] p_full[2]
-//   o_done[2] drain claim item_full[4] item_empty[4] p_half[2]
+//   o_done[2] drain claim item_full[4] item_empty[4]
 // then 4 item slots (idx, mb, kvz, bh, n0, n1), the TMEM slot and the abort flag.
 template <int D, bool BYTE>
 struct FwdPersistCfg : FwdCfg<D, BYTE> {
@@ -28,7 +28,7 @@ struct FwdPersistCfg : FwdCfg<D, BYTE> {
   static_assert(!Base::PSMEM, "the persistent kernel keeps P in tensor memory");
   static constexpr int ITEM_RING = 4;
   static constexpr int ITEM_INTS = 6;
-  static constexpr int NBAR = 4 + 2 * Base::KSTAGES + 2 * Base::VSTAGES + 6 + 2 + 2 * ITEM_RING + 2;
+  static constexpr int NBAR = 4 + 2 * Base::KSTAGES + 2 * Base::VSTAGES + 6 + 2 + 2 * ITEM_RING;
   static constexpr int SMEM_USED = Base::OFF_BAR + NBAR * 8 + ITEM_RING * ITEM_INTS * 4 + 32;
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 120 * 1024 ? (SMEM_USED + 1024) : 120 * 1024;
   static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
@@ -103,9 +103,7 @@ __global__ void __launch_bounds__(FwdRoles<false>::kThreads, 1)
   uint64_t* claim = drain + 1;  // the K/V loads of an item are all issued: take the next item
   uint64_t* item_full = claim + 1;
   uint64_t* item_empty = item_full + C::ITEM_RING;
-  uint64_t* p_half = item_empty + C::ITEM_RING;  // P released in halves only
-  volatile int* item_slot = reinterpret_cast<volatile int*>(p_half + 2);
-  constexpr bool PS = TATTN_PSPLIT != 0;
+  volatile int* item_slot = reinterpret_cast<volatile int*>(item_empty + C::ITEM_RING);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(item_slot) + C::ITEM_RING * C::ITEM_INTS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -118,7 +116,6 @@ __global__ void __launch_bounds__(FwdRoles<false>::kThreads, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], TATTN_PFULL_PER_WARP ? R::kThreadsPerTile / 32 : R::kThreadsPerTile);
       mbar_init(&o_done[i], 1);
-      mbar_init(&p_half[i], R::kThreadsPerTile / 32);
     }
     for (int i = 0; i < C::KSTAGES; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < C::VSTAGES; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
@@ -302,23 +299,14 @@ __global__ void __launch_bounds__(FwdRoles<false>::kThreads, 1)
           const int ks1 = (g + j + 1) % C::KSTAGES;
           for (int t = 0; t < 2 && ok; ++t) {
             if (j >= n_of(t)) continue;
-            const uint32_t pph = pc[t] & 1;
-            if (!(ok = mbar_wait(PS ? &p_half[t] : &p_full[t], pph, abort_flag, W_MMA + 3))) break;
+            if (!(ok = mbar_wait(&p_full[t], pc[t] & 1, abort_flag, W_MMA + 3))) break;
             ++pc[t];
             tc_fence_after();
             if (users_first(j) == t) {
               if (!(ok = mbar_wait(&v_full[vs], ((g + j) / C::VSTAGES) & 1, abort_flag, W_MMA + 4))) break;
               tc_fence_after();
             }
-            if constexpr (PS) {
-              // keys 0..63 of the tile as soon as their P is in, the rest once all of P is
-              issue_pv<D, FP16, 0, 4>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
-              if (!(ok = mbar_wait(&p_full[t], pph, abort_flag, W_MMA + 6))) break;
-              tc_fence_after();
-              issue_pv<D, FP16, 4, 8>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, true);
-            } else {
-              issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
-            }
+            issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
             if (j + 1 == n_of(t)) mma_commit(&o_done[t]);  // the tile's last P V: O is final
             if (users_last(j) == t) mma_commit(&v_empty[vs]);
             if (j + 1 < n_of(t)) {
@@ -389,11 +377,9 @@ __global__ void __launch_bounds__(FwdRoles<false>::kThreads, 1)
         const bool diag = p.causal && (j == nt - 1);
         if (diag || (col0 + 128 > p.Nk)) {
           const int lim = (diag ? min(row + 1, p.Nk) : p.Nk) - col0;
-          ok = softmax_step<D, QK, FP16, true, PS>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag,
-                                                   &p_half[t]);
+          ok = softmax_step<D, QK, FP16, true>(tS, tO, sc, lim, j, m_run, l_run, &o_done[t], abort_flag);
         } else {
-          ok = softmax_step<D, QK, FP16, false, PS>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag,
-                                                    &p_half[t]);
+          ok = softmax_step<D, QK, FP16, false>(tS, tO, sc, 128, j, m_run, l_run, &o_done[t], abort_flag);
         }
         if (!ok) break;
         tmem_st_wait();
