@@ -198,11 +198,15 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint3
   constexpr uint32_t idesc = INT8             ? instr_desc(2, 1, 0, 0, 128, 128)
                              : QK == QK_F8 ? instr_desc(1, 0, 0, 0, 128, 128)  // E4M3 x E4M3 -> F32
                                            : instr_desc(1, FP16 ? 0 : 1, 0, 0, 128, 128);
+  // one descriptor per operand; each K step adds its byte offset / 16 to the start-address field
+  // (addresses stay below 256 KB, so the 14-bit field never carries)
+  const uint64_t ad0 = smem_desc(q_smem, 16, 8 * C::QK_SPAN, C::QK_SWZ);
+  const uint64_t bd0 = smem_desc(k_smem, 16, 8 * C::QK_SPAN, C::QK_SWZ);
 #pragma unroll
   for (int kk = 0; kk < C::QK_STEPS; ++kk) {
     const uint32_t off = (uint32_t)((kk * 32) / C::QK_SPAN) * C::QK_PANEL_BYTES + (uint32_t)((kk * 32) % C::QK_SPAN);
-    const uint64_t ad = smem_desc(q_smem + off, 16, 8 * C::QK_SPAN, C::QK_SWZ);
-    const uint64_t bd = smem_desc(k_smem + off, 16, 8 * C::QK_SPAN, C::QK_SWZ);
+    const uint64_t ad = ad0 + (off >> 4);
+    const uint64_t bd = bd0 + (off >> 4);
     if constexpr (INT8)
       mma_i8_ss(s_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
     else if constexpr (QK == QK_F8)
@@ -216,11 +220,12 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_smem, uint3
 template <int D, bool FP16>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
   constexpr uint32_t idesc = instr_desc(1, FP16 ? 0 : 1, 0, 1, 128, D);
+  // 16 keys per step = 16 rows of 128 B; 64-column panels of V are 128 x 128 B apart (LBO),
+  // groups of 8 key rows are 1024 B apart (SBO).  One descriptor; each step adds 2 KB / 16.
+  const uint64_t bd0 = smem_desc(v_smem, 128 * 128, 1024, kSwizzle128B);
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk) {
-    // 16 keys per step = 16 rows of 128 B; 64-column panels of V are 128 x 128 B apart (LBO),
-    // groups of 8 key rows are 1024 B apart (SBO).
-    const uint64_t bd = smem_desc(v_smem + kk * 16 * 128, 128 * 128, 1024, kSwizzle128B);
+    const uint64_t bd = bd0 + (uint64_t)(kk * 16 * 128 / 16);
     mma_f16_ts(o_tmem, p_tmem + kk * 8, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -895,20 +900,18 @@ __global__ void __launch_bounds__(FwdRoles<SPLIT>::kThreads, 1)
         const int ks1 = (j + 1) % C::KSTAGES;
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= n_of(t)) continue;
+          // V(j) and K(j + 1) first (normally loaded long before), then P: once P is in, P V and
+          // the next Q K^T go out with no further wait in between
+          if (users_first(j) == t)
+            if (!(ok = mbar_wait(&v_full[vs], (j / C::VSTAGES) & 1, abort_flag, W_MMA + 4))) break;
+          if (j + 1 < n_of(t) && users_first(j + 1) == t)
+            if (!(ok = mbar_wait(&k_full[ks1], ((j + 1) / C::KSTAGES) & 1, abort_flag, W_MMA + 5))) break;
           if (!(ok = mbar_wait(&p_full[t], j & 1, abort_flag, W_MMA + 3))) break;
           tc_fence_after();
-          if (users_first(j) == t) {
-            if (!(ok = mbar_wait(&v_full[vs], (j / C::VSTAGES) & 1, abort_flag, W_MMA + 4))) break;
-            tc_fence_after();
-          }
           issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
           if (j + 1 == n_of(t)) mma_commit(&o_done[t]);  // the tile's last P V: O is final
           if (users_last(j) == t) mma_commit(&v_empty[vs]);
           if (j + 1 < n_of(t)) {
-            if (users_first(j + 1) == t) {
-              if (!(ok = mbar_wait(&k_full[ks1], ((j + 1) / C::KSTAGES) & 1, abort_flag, W_MMA + 5))) break;
-              tc_fence_after();
-            }
             issue_qk<D, QK, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr + ks1 * C::K_TILE);
             mma_commit(&s_full[t]);
             if (users_last(j + 1) == t) mma_commit(&k_empty[ks1]);

@@ -299,21 +299,18 @@ __global__ void __launch_bounds__(FwdRoles<false>::kThreads, 1)
           const int ks1 = (g + j + 1) % C::KSTAGES;
           for (int t = 0; t < 2 && ok; ++t) {
             if (j >= n_of(t)) continue;
+            // V(j) and K(j + 1) first (normally loaded long before), then P
+            if (users_first(j) == t)
+              if (!(ok = mbar_wait(&v_full[vs], ((g + j) / C::VSTAGES) & 1, abort_flag, W_MMA + 4))) break;
+            if (j + 1 < n_of(t) && users_first(j + 1) == t)
+              if (!(ok = mbar_wait(&k_full[ks1], ((g + j + 1) / C::KSTAGES) & 1, abort_flag, W_MMA + 5))) break;
             if (!(ok = mbar_wait(&p_full[t], pc[t] & 1, abort_flag, W_MMA + 3))) break;
             ++pc[t];
             tc_fence_after();
-            if (users_first(j) == t) {
-              if (!(ok = mbar_wait(&v_full[vs], ((g + j) / C::VSTAGES) & 1, abort_flag, W_MMA + 4))) break;
-              tc_fence_after();
-            }
             issue_pv<D, FP16>(tmem + C::tm_o(t), tmem + C::tm_s(t), v_addr + vs * C::V_TILE, j > 0);
             if (j + 1 == n_of(t)) mma_commit(&o_done[t]);  // the tile's last P V: O is final
             if (users_last(j) == t) mma_commit(&v_empty[vs]);
             if (j + 1 < n_of(t)) {
-              if (users_first(j + 1) == t) {
-                if (!(ok = mbar_wait(&k_full[ks1], ((g + j + 1) / C::KSTAGES) & 1, abort_flag, W_MMA + 5))) break;
-                tc_fence_after();
-              }
               issue_qk<D, QK, FP16>(tmem + C::tm_s(t), q_addr + t * C::Q_TILE, k_addr + ks1 * C::K_TILE);
               mma_commit(&s_full[t]);
               if (j + 2 == n_of(t)) mma_commit(&q_empty[t]);  // the tile's last Q K^T of this item
