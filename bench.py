@@ -709,6 +709,48 @@ def _prepass_bytes(w):
     return 3 * nk + 3 * nq + 4 * w.B * w.Hq * w.N
 
 
+def run_fused_sweep(args):
+    """The fused kernels alone on the 4096-, 8192-, 16384- and 131072-token workloads, every mode:
+    one JSON line per (workload, mode) with the fused kernel's time and TFLOP/s (CUDA events, back
+    to back, after 3 warm-ups; inputs larger than L2).  With --lib this times a variant build."""
+    import tiled_attention_22_b200 as ta
+
+    for cfg in (2, 3, 4, 5):
+        w = WORKLOADS[cfg]
+        q, k, v = (t.cuda() for t in make_inputs(w))
+        reps = 3 if cfg == 5 else 20
+        for mode in [m for m in ("int8_qk", "bf16_exact", "fp8_qk") if m in args.modes.split(",")]:
+            if mode == "bf16_exact":
+                o, l = ta.attn_fwd(q, k, v, causal=w.causal)
+
+                def fn():
+                    ta.attn_fwd(q, k, v, causal=w.causal, out=o, lse=l)
+            else:
+                quant = ta.attn_quant_smooth_k if mode == "int8_qk" else ta.attn_quant_smooth_k_fp8
+                fused = ta.attn_fwd_int8_quantized if mode == "int8_qk" else ta.attn_fwd_fp8_quantized
+                pre = quant(q, k)
+                o, l = fused(pre, v, causal=w.causal)
+
+                def fn():
+                    fused(pre, v, causal=w.causal, out=o, lse=l)
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if ta.attn_check_status() != 0:
+                raise RuntimeError("device-side wait timed out in the fused-kernel sweep")
+            ms = e0.elapsed_time(e1) / reps
+            print(json.dumps({"lib": args.lib or "in-tree", "workload": w.name, "mode": mode, "fused_ms": ms,
+                              "tflops": w.flops() / ms / 1e9}), flush=True)
+        del q, k, v
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -721,12 +763,22 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the measurements of the other paths (KV-cache decode, prefix mask, ring)")
     ap.add_argument("--no-others", action="store_true", help="skip the other workloads (N = 4096, 8192, 16384)")
     ap.add_argument("--no-gemm-peaks", action="store_true", help="skip timing the 8-bit library GEMMs")
+    ap.add_argument("--lib", default=None, help="load this build of the library (a variant from build.py --out)")
+    ap.add_argument("--fused-sweep", action="store_true",
+                    help="time only the fused kernels on the N >= 4096 workloads (one JSON line each)")
     ap.add_argument("--modes", default="int8_qk,bf16_exact,fp8_qk",
                     help="modes to time (the headline value is int8_qk; drop one only for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.config]
+    if args.lib:
+        from tiled_attention_22_b200 import binding
+
+        binding.load_library(args.lib)
+    if args.fused_sweep:
+        run_fused_sweep(args)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -35,20 +35,35 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(os.path.join(HERE, d)) <= t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, defines=(), out: str = None) -> str:
+    """Build the library.  ``defines`` ("NAME=VALUE" strings) select compile-time variants of the
+    kernels (the measurement variants named in the kernel sources); a variant build goes to
+    ``out`` and never replaces the in-tree library."""
+    target = out or LIB_PATH
+    if not force and not defines and out is None and up_to_date():
         return LIB_PATH
-    os.makedirs(LIB_DIR, exist_ok=True)
+    os.makedirs(os.path.dirname(os.path.abspath(target)), exist_ok=True)
     cmd = [nvcc(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
            "-shared", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"),
-           "-I", os.path.join(HERE, "csrc"), "-o", LIB_PATH + ".tmp"]
+           "-I", os.path.join(HERE, "csrc"), "-o", target + ".tmp"]
+    cmd += [f"-D{d}" for d in defines]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(HERE, s) for s in SOURCES]
     subprocess.run(cmd, check=True)
-    os.replace(LIB_PATH + ".tmp", LIB_PATH)
-    return LIB_PATH
+    os.replace(target + ".tmp", target)
+    return target
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    import argparse
+
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("-v", action="store_true", help="ptxas register / spill report")
+    ap.add_argument("--define", action="append", default=[], help="NAME=VALUE for a kernel variant (repeatable)")
+    ap.add_argument("--out", default=None, help="output path for a variant build")
+    a = ap.parse_args()
+    if a.define and not a.out:
+        ap.error("a variant build (--define) needs --out")
+    print(build(force=a.force, verbose=a.v, defines=a.define, out=a.out))
