@@ -113,6 +113,19 @@ int launch_quant(const uint16_t* q16, const uint16_t* k16, int B, int Hq, int Hk
   return ATTN_OK;
 }
 
+// Once per device and kernel: allow `bytes` of dynamic shared memory.
+template <class Kern>
+int allow_dynamic_smem(Kern kern, int bytes, std::atomic<int>* done) {
+  int dev = 0;
+  TATTN_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_LAUNCH;
+  if (done[dev].load(std::memory_order_acquire) != 1) {
+    TATTN_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+    done[dev].store(1, std::memory_order_release);
+  }
+  return ATTN_OK;
+}
+
 // The pre-pass: K channel mean (float64 partials, then the final division), then smoothing and
 // quantisation of K and quantisation of Q with the lse bias; f8 selects E4M3 codes over INT8.
 int launch_prepass(const void* q, const void* k, int B, int Hq, int Hkv, int N, int d, int dtype, float scale,
@@ -134,7 +147,17 @@ int launch_prepass(const void* q, const void* k, int B, int Hq, int Hkv, int N, 
     }
     TATTN_CUDA(cudaGetLastError());
   }
-  kmean_final_kernel<<<(BG * d + 127) / 128, 128, 0, stream>>>(part, BG, N, d, kmean);
+  if (d == 128) {
+    static std::atomic<int> set128[kMaxDevices];
+    int rc = allow_dynamic_smem(kmean_final_kernel<128>, kmean_final_smem<128>(), set128);
+    if (rc) return rc;
+    kmean_final_kernel<128><<<BG, kFinalThreads, kmean_final_smem<128>(), stream>>>(part, N, kmean);
+  } else {
+    static std::atomic<int> set64[kMaxDevices];
+    int rc = allow_dynamic_smem(kmean_final_kernel<64>, kmean_final_smem<64>(), set64);
+    if (rc) return rc;
+    kmean_final_kernel<64><<<BG, kFinalThreads, kmean_final_smem<64>(), stream>>>(part, N, kmean);
+  }
   TATTN_CUDA(cudaGetLastError());
   const unsigned qblocks = (unsigned)((long long)B * Hkv * T + (long long)B * Hq * T);
   return f8 ? launch_quant<true>(q16, k16, B, Hq, Hkv, N, d, fp16, scale, kmean, q8, sq, k8, sk, bias, qblocks, stream)

@@ -11,7 +11,8 @@
 // These kernels are HBM-bound: plain 16-byte vector loads and stores, no tensor cores.
 //   kmean_partial_kernel  K -> float64 partial sums per 128-token block (sequential in token order,
 //                         the block staged in shared memory)
-//   kmean_final_kernel    partials -> mean (sequential in block order), (float)(total / N)
+//   kmean_final_kernel    partials -> mean (sequential in block order), (float)(total / N); the
+//                         partials stream through shared memory (cp.async pipeline)
 //   quant_kernel          K blocks: smooth + quantise -> k8, sk;  Q blocks: quantise -> q8, sq and
 //                         the lse bias scale * q_i . mean (row dot product, warp-shuffle reduced)
 #pragma once
@@ -79,17 +80,62 @@ __global__ void __launch_bounds__(D) kmean_partial_kernel(const uint16_t* __rest
   part[((size_t)bg * T + t) * D + c] = acc;
 }
 
-// One thread = one (batch*kv head, channel): total over blocks in ascending order, then the mean.
-__global__ void __launch_bounds__(128) kmean_final_kernel(const double* __restrict__ part, int BG, int N, int d,
-                                                           float* __restrict__ kmean) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= BG * d) return;
-  const int bg = idx / d, c = idx % d;
+// One CTA per (batch * kv head): thread c < D adds channel c's block partials in ascending block
+// order into a float64 total, then writes (float)(total / N).  The partials of one (batch, kv head)
+// ([T][D] float64, contiguous) stream through shared memory in chunks of kFinalChunk blocks with
+// cp.async, kFinalStages - 1 chunks in flight, so the sequential adds never wait on a global load.
+constexpr int kFinalThreads = 512;
+constexpr int kFinalChunk = 16;
+constexpr int kFinalStages = 8;
+template <int D>
+constexpr int kmean_final_smem() { return kFinalStages * kFinalChunk * D * (int)sizeof(double); }
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int D>
+__global__ void __launch_bounds__(kFinalThreads) kmean_final_kernel(const double* __restrict__ part, int N,
+                                                                     float* __restrict__ kmean) {
+  extern __shared__ __align__(16) double fbuf[];  // [kFinalStages][kFinalChunk * D]
+  constexpr int CHUNK = kFinalChunk * D;        // doubles per chunk
+  const int bg = blockIdx.x;
   const int T = (N + 127) / 128;
-  const double* src = part + (size_t)bg * T * d + c;
+  const double* src = part + (size_t)bg * T * D;
+  const int total_elems = T * D;
+  const int nchunk = (T + kFinalChunk - 1) / kFinalChunk;
+  // chunk k -> stage k % kFinalStages; each thread copies 16-byte pieces (two partials)
+  auto issue = [&](int k) {
+    if (k < nchunk) {
+      double* dst = fbuf + (k % kFinalStages) * CHUNK;
+      const int base = k * CHUNK;
+      for (int e = 2 * threadIdx.x; e < CHUNK; e += 2 * kFinalThreads)
+        if (base + e < total_elems) cp_async16(dst + e, src + base + e);
+    }
+    cp_async_commit();  // one group per chunk (empty past the end), so group counts stay aligned
+  };
+#pragma unroll 1
+  for (int k = 0; k < kFinalStages - 1; ++k) issue(k);
   double total = 0.0;
-  for (int t = 0; t < T; ++t) total = __dadd_rn(total, src[(size_t)t * d]);
-  kmean[idx] = __double2float_rn(__ddiv_rn(total, (double)N));
+#pragma unroll 1
+  for (int k = 0; k < nchunk; ++k) {
+    cp_async_wait<kFinalStages - 2>();  // chunk k has landed (this thread's copies)
+    __syncthreads();                    // ... and every other thread's
+    if (threadIdx.x < D) {
+      const double* b = fbuf + (k % kFinalStages) * CHUNK + threadIdx.x;
+      const int nt = min(kFinalChunk, T - k * kFinalChunk);
+      for (int t = 0; t < nt; ++t) total = __dadd_rn(total, b[t * D]);
+    }
+    __syncthreads();                    // stage k % kFinalStages is free again
+    issue(k + kFinalStages - 1);
+  }
+  cp_async_wait<0>();
+  if (threadIdx.x < D) kmean[(size_t)bg * D + threadIdx.x] = __double2float_rn(__ddiv_rn(total, (double)N));
 }
 
 // One CTA per 128-token block (4*D threads: 512 for d=128, 256 for d=64).  Blocks [0, nK) are K
