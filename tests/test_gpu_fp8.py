@@ -13,6 +13,7 @@ import torch
 import oracle
 from attn_workloads import WORKLOADS, Workload, make_inputs
 from oracle import fp8_emulation as f8
+from sampling import boundary_rows, sample_heads
 from tolerances import INT8_COS as Q_COS, INT8_LSE as Q_LSE, INT8_MAX as Q_MAX, assert_close16, quant_metrics
 
 pytestmark = pytest.mark.gpu
@@ -113,12 +114,6 @@ def test_fp8_fwd_equals_prepass_plus_fused(ta):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-def _sample_rows(N, rng, n=12):
-    rows = {0, 1, min(127, N - 1), min(128, N - 1), N - 1, N // 2}
-    rows |= set(rng.integers(0, N, n).tolist())
-    return sorted(rows)
-
-
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
 def test_fp8_full_size_sampled_rows(ta, cfg):
     w = WORKLOADS[cfg]
@@ -128,9 +123,9 @@ def test_fp8_full_size_sampled_rows(ta, cfg):
     assert ta.attn_check_status() == 0
     rng = np.random.default_rng(cfg + 50)
     G = w.Hq // w.Hkv
-    for b, h in [(0, 0), (w.B - 1, w.Hq - 1), (int(rng.integers(w.B)), int(rng.integers(w.Hq)))]:
+    rows = boundary_rows(w.N, rng)
+    for b, h in sample_heads(w.B, w.Hq, w.Hkv, rng):
         g = h // G
-        rows = _sample_rows(w.N, rng)
         qs, ks, vs = q[b:b + 1, h:h + 1], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1]
         og = _np(o[b, h, rows])[None, None]
         lg = l[b, h, rows].cpu().numpy().astype(np.float64)[None, None]

@@ -23,6 +23,7 @@ import torch
 
 import oracle
 from attn_workloads import WORKLOADS, Workload, make_inputs
+from sampling import boundary_rows, sample_heads
 from tolerances import (BF16_LSE, BF16_MAX, INT8_COS, INT8_LSE, INT8_MAX, assert_close16, cosine, max_excess,
                         quant_metrics)
 
@@ -164,17 +165,13 @@ def test_int32_scores_bit_exact(ta, d):
         np.testing.assert_array_equal(out[i], want, err_msg=str((b, h, m, n)))
 
 
-def _sample_rows(N, rng, n=12):
-    rows = {0, 1, min(127, N - 1), min(128, N - 1), N - 1, N // 2}
-    rows |= set(rng.integers(0, N, n).tolist())
-    return sorted(rows)
-
-
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
 @pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk"])
 def test_full_size_sampled_rows(ta, cfg, mode):
     """The named workloads at full size, in the launch configuration the benchmark times; the oracle
-    computes sampled rows of sampled heads (rows are independent, so this is exact for them)."""
+    computes sampled rows of sampled heads (rows are independent, so this is exact for them): every
+    query-tile and work-item boundary near the start, middle and end, the last rows, random rows,
+    and heads on both sides of a GQA group boundary (tests/sampling.py)."""
     w = WORKLOADS[cfg]
     q, k, v = make_inputs(w)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
@@ -183,11 +180,11 @@ def test_full_size_sampled_rows(ta, cfg, mode):
     assert ta.attn_check_status() == 0
     rng = np.random.default_rng(cfg)
     G = w.Hq // w.Hkv
-    heads = [(0, 0), (w.B - 1, w.Hq - 1), (int(rng.integers(w.B)), int(rng.integers(w.Hq)))]
+    heads = sample_heads(w.B, w.Hq, w.Hkv, rng)
+    rows = boundary_rows(w.N, rng)
     o_all, O_all, Oe_all = [], [], []
     for b, h in heads:
         g = h // G
-        rows = _sample_rows(w.N, rng)
         qs, ks, vs = q[b:b + 1, h:h + 1], k[b:b + 1, g:g + 1], v[b:b + 1, g:g + 1]
         og = _np(o[b, h, rows])[None, None]
         lg = l[b, h, rows].cpu().numpy().astype(np.float64)[None, None]
