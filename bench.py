@@ -736,6 +736,8 @@ def run_fused_sweep(args):
             for _ in range(3):
                 fn()
             torch.cuda.synchronize()
+            if ta.attn_check_status() != 0:  # stop before timing a build whose waits run out
+                raise RuntimeError(f"device-side wait timed out ({w.name}, {mode})")
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             for _ in range(reps):
