@@ -216,12 +216,16 @@ int attn_probe_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int H
  * attn_fwd_host - attn_fwd with HOST buffers: copies q, k, v from host memory into the caller's
  * device buffers dq, dk, dv, runs the forward pass into do_ / dlse, and copies o (and lse when
  * both lse pointers are non-NULL) back to host memory; returns when the host outputs are ready.
- * The work is split into up to 8 chunks of whole (batch, kv head) units: chunk c's inputs are
- * copied in on a helper stream while earlier chunks compute on `stream`, and outputs are copied
- * out on a second helper stream (two streams and per-chunk events are created and destroyed by
- * the call; no device memory is allocated).  Host buffers should be pinned for the copies to
- * overlap.  One cudaMemcpyAsync per buffer per chunk.  INT8 mode needs workspace of at least
- * attn_workspace_bytes(B,Hq,Hkv,N,d,mode) bytes (chunks reuse it in turn).
+ * The work is split into at most 10 pieces, each a run of query heads: piece c's inputs are
+ * copied in on a helper stream while earlier pieces compute on `stream`, and outputs are copied
+ * out on a second helper stream (two streams and per-piece events are created and destroyed by
+ * the call; no device memory is allocated).  When N % 4 == 0 the first and last pieces are one
+ * query head each (one (batch, kv head) unit when Hq == Hkv), so that little copying is left
+ * outside the compute; the (batch, kv head) units between them form up to six pieces.  Otherwise
+ * the pieces are up to 8 runs of whole units.  Outputs are bit-identical to attn_fwd's.  Host
+ * buffers should be pinned for the copies to overlap.  One cudaMemcpyAsync per buffer per piece.
+ * The 8-bit modes need workspace of at least attn_workspace_bytes(B,Hq,Hkv,N,d,mode) bytes (pieces
+ * reuse it in turn).
  */
 int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
                   void* dq, void* dk, void* dv, void* do_, float* dlse,

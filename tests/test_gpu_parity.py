@@ -272,10 +272,12 @@ def test_canaries_around_outputs(ta, mode):
     assert torch.isfinite(o).all() and torch.isfinite(l).all()
 
 
-@pytest.mark.parametrize("shape", [(1, 4, 2, 500, 128), (3, 6, 3, 333, 64), (2, 8, 8, 1024, 128)])
+@pytest.mark.parametrize("shape", [(1, 4, 2, 500, 128), (3, 6, 3, 333, 64), (2, 8, 8, 1024, 128), (1, 4, 1, 256, 128),
+                                   (2, 8, 2, 2048, 64)])
 def test_host_buffer_entry_point_matches_device_call(ta, shape):
-    """attn_fwd_host pipelines copies and compute over chunks of (batch, kv head) units; its host
-    outputs must equal the device call's bit for bit (odd N exercises 4-unit-aligned chunks)."""
+    """attn_fwd_host pipelines copies and compute over pieces of query heads (single heads at both
+    ends, runs of (batch, kv head) units between, or whole units only when N % 4 != 0); its host
+    outputs must equal the device call's bit for bit (odd N exercises 4-unit-aligned pieces)."""
     B, Hq, Hkv, N, d = shape
     w = Workload("t", B, Hq, Hkv, N, d, True, "bf16", "k_offset", 99500 + N)
     q, k, v = make_inputs(w)

@@ -392,18 +392,52 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool want_lse = lse && dlse;
   // Units are (batch, kv head) pairs with their G query heads: independent problems whose Q, K, V,
-  // O and lse slices are contiguous, in unit order, in every [B, H, N, d] tensor.  A run of units
-  // is therefore one contiguous problem with B' = 1, Hq' = n*G, Hkv' = n.  The units are split
-  // into chunks; chunk c's inputs are copied in on a helper stream while chunk c-1 computes on
-  // the caller's stream, and its outputs are copied out on a second helper stream.
+  // O and lse slices are contiguous, in unit order, in every [B, H, N, d] tensor.  A run of whole
+  // units is one problem with B' = 1, Hq' = n*G, Hkv' = n, and a run of query heads inside one
+  // unit is one with B' = 1, Hq' = n, Hkv' = 1 (the unit's K and V); either gives every output row
+  // the same arithmetic as the whole call.  The work is cut into pieces of query heads; piece c's
+  // inputs are copied in on a helper stream while piece c-1 computes on the caller's stream, and
+  // its outputs are copied out on a second helper stream.  Only the first piece's input copy and
+  // the last piece's output copy are not hidden behind compute, so when every head's lse slice is
+  // 16-byte aligned (N % 4 == 0) the first and last pieces are a single query head (a single unit
+  // when G = 1) and the units between them form up to six pieces.  Otherwise pieces are up to 8
+  // runs of whole units, 4-unit aligned when a unit's lse slice is not 16-byte aligned.
   const int G = Hq / Hkv;
-  const int units = B * Hkv;
-  const int nchunk = units < 8 ? units : 8;
-  const size_t q_unit = (size_t)G * N * d * 2, kv_unit = (size_t)N * d * 2, l_unit = (size_t)G * N * 4;
+  const int units = B * Hkv, heads = B * Hq;
+  const size_t q_head = (size_t)N * d * 2, kv_unit = (size_t)N * d * 2, l_head = (size_t)N * 4;
+  constexpr int kMaxPieces = 16;
+  int cut[kMaxPieces + 1];
+  int npiece = 0;
+  {
+    int c[kMaxPieces + 8];
+    int nc = 0;
+    if (N % 4 == 0) {
+      c[nc++] = 0;
+      c[nc++] = 1;
+      c[nc++] = G;
+      const int mid = units - 2 > 0 ? units - 2 : 0;  // units strictly between the first and last
+      const int nm = mid < 6 ? mid : 6;
+      for (int i = 1; i < nm; ++i) c[nc++] = (1 + (int)((long long)mid * i / nm)) * G;
+      c[nc++] = heads - G;
+      c[nc++] = heads - 1;
+      c[nc++] = heads;
+    } else {
+      const int align_units = ((size_t)G * l_head % 16 == 0) ? 1 : 4;
+      const int n8 = units < 8 ? units : 8;
+      for (int i = 0; i <= n8; ++i) c[nc++] = (int)((long long)units * i / n8) / align_units * align_units * G;
+      c[nc++] = heads;
+    }
+    std::sort(c, c + nc);
+    for (int i = 0; i < nc; ++i) {
+      if (i > 0 && c[i] == c[i - 1]) continue;
+      cut[npiece++] = c[i];
+    }
+    npiece -= 1;  // cut[0..npiece] bound npiece pieces
+  }
   cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t ev_in[8] = {}, ev_done[8] = {};
+  cudaEvent_t ev_in[kMaxPieces] = {}, ev_done[kMaxPieces] = {};
   auto cleanup = [&]() {
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < kMaxPieces; ++c) {
       if (ev_in[c]) cudaEventDestroy(ev_in[c]);
       if (ev_done[c]) cudaEventDestroy(ev_done[c]);
     }
@@ -420,40 +454,38 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   } while (0)
   TATTN_CUDA_C(cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking));
   TATTN_CUDA_C(cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking));
-  for (int c = 0; c < nchunk; ++c) {
+  for (int c = 0; c < npiece; ++c) {
     TATTN_CUDA_C(cudaEventCreateWithFlags(&ev_in[c], cudaEventDisableTiming));
     TATTN_CUDA_C(cudaEventCreateWithFlags(&ev_done[c], cudaEventDisableTiming));
   }
   // inputs may still be in use by earlier work on the caller's stream: start after it
   TATTN_CUDA_C(cudaEventRecord(ev_done[0], st));
   TATTN_CUDA_C(cudaStreamWaitEvent(s_in, ev_done[0], 0));
-  // lse slices must stay 16-byte aligned: 4 units always are (4 * G * N * 4 bytes)
-  const int align_units = (l_unit % 16 == 0) ? 1 : 4;
-  auto chunk_begin = [&](int c) {
-    if (c >= nchunk) return units;
-    return (int)((long long)units * c / nchunk) / align_units * align_units;
+  auto copy_in = [&](size_t off, size_t bytes, void* dst, const void* src) {
+    return cudaMemcpyAsync(static_cast<uint8_t*>(dst) + off, static_cast<const uint8_t*>(src) + off, bytes,
+                           cudaMemcpyHostToDevice, s_in);
   };
-  for (int c = 0; c < nchunk; ++c) {
-    const int u0 = chunk_begin(c), n = chunk_begin(c + 1) - u0;
-    if (n <= 0) continue;
-    TATTN_CUDA_C(cudaMemcpyAsync(static_cast<uint8_t*>(dq) + u0 * q_unit, static_cast<const uint8_t*>(q) + u0 * q_unit,
-                                 n * q_unit, cudaMemcpyHostToDevice, s_in));
-    TATTN_CUDA_C(cudaMemcpyAsync(static_cast<uint8_t*>(dk) + u0 * kv_unit,
-                                 static_cast<const uint8_t*>(k) + u0 * kv_unit, n * kv_unit, cudaMemcpyHostToDevice,
-                                 s_in));
-    TATTN_CUDA_C(cudaMemcpyAsync(static_cast<uint8_t*>(dv) + u0 * kv_unit,
-                                 static_cast<const uint8_t*>(v) + u0 * kv_unit, n * kv_unit, cudaMemcpyHostToDevice,
-                                 s_in));
+  for (int c = 0; c < npiece; ++c) {
+    const int h0 = cut[c], h1 = cut[c + 1];
+    TATTN_CUDA_C(copy_in(h0 * q_head, (size_t)(h1 - h0) * q_head, dq, q));
+    // K and V of every unit this piece starts (a piece inside a unit that another piece started
+    // reuses them)
+    const int u0 = (h0 + G - 1) / G, u1 = (h1 + G - 1) / G;
+    if (u1 > u0) {
+      TATTN_CUDA_C(copy_in(u0 * kv_unit, (size_t)(u1 - u0) * kv_unit, dk, k));
+      TATTN_CUDA_C(copy_in(u0 * kv_unit, (size_t)(u1 - u0) * kv_unit, dv, v));
+    }
     TATTN_CUDA_C(cudaEventRecord(ev_in[c], s_in));
   }
-  for (int c = 0; c < nchunk; ++c) {
-    const int u0 = chunk_begin(c), n = chunk_begin(c + 1) - u0;
-    if (n <= 0) continue;
+  for (int c = 0; c < npiece; ++c) {
+    const int h0 = cut[c], h1 = cut[c + 1];
+    const bool whole = h0 % G == 0 && (h1 - h0) % G == 0;
+    const int hq = h1 - h0, hkv = whole ? hq / G : 1, ukv = h0 / G;
     TATTN_CUDA_C(cudaStreamWaitEvent(st, ev_in[c], 0));
-    rc = attn_fwd(static_cast<uint8_t*>(dq) + u0 * q_unit, static_cast<uint8_t*>(dk) + u0 * kv_unit,
-                  static_cast<uint8_t*>(dv) + u0 * kv_unit, static_cast<uint8_t*>(do_) + u0 * q_unit,
-                  want_lse ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(dlse) + u0 * l_unit) : nullptr, 1,
-                  n * G, n, N, d, causal, scale, mode, dtype, workspace, ws_bytes, stream);
+    rc = attn_fwd(static_cast<uint8_t*>(dq) + h0 * q_head, static_cast<uint8_t*>(dk) + ukv * kv_unit,
+                  static_cast<uint8_t*>(dv) + ukv * kv_unit, static_cast<uint8_t*>(do_) + h0 * q_head,
+                  want_lse ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(dlse) + h0 * l_head) : nullptr, 1,
+                  hq, hkv, N, d, causal, scale, mode, dtype, workspace, ws_bytes, stream);
     if (rc) {
       cudaStreamSynchronize(s_in);
       cudaStreamSynchronize(st);
@@ -462,12 +494,12 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
     }
     TATTN_CUDA_C(cudaEventRecord(ev_done[c], st));
     TATTN_CUDA_C(cudaStreamWaitEvent(s_out, ev_done[c], 0));
-    TATTN_CUDA_C(cudaMemcpyAsync(static_cast<uint8_t*>(o) + u0 * q_unit, static_cast<uint8_t*>(do_) + u0 * q_unit,
-                                 n * q_unit, cudaMemcpyDeviceToHost, s_out));
+    TATTN_CUDA_C(cudaMemcpyAsync(static_cast<uint8_t*>(o) + h0 * q_head, static_cast<uint8_t*>(do_) + h0 * q_head,
+                                 (size_t)hq * q_head, cudaMemcpyDeviceToHost, s_out));
     if (want_lse)
-      TATTN_CUDA_C(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(lse) + u0 * l_unit,
-                                   reinterpret_cast<uint8_t*>(dlse) + u0 * l_unit, n * l_unit, cudaMemcpyDeviceToHost,
-                                   s_out));
+      TATTN_CUDA_C(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(lse) + h0 * l_head,
+                                   reinterpret_cast<uint8_t*>(dlse) + h0 * l_head, (size_t)hq * l_head,
+                                   cudaMemcpyDeviceToHost, s_out));
   }
   TATTN_CUDA_C(cudaStreamSynchronize(s_out));
   TATTN_CUDA_C(cudaStreamSynchronize(st));
