@@ -393,6 +393,11 @@ class _Modes:
         return {"ms_total": ms, "ms_per_step": ms / steps, "tflops": tflops, "kernel_ms": kern}
 
 
+# Datasheet dense tensor peaks of one B200 (TFLOP/s; NVIDIA's sparse figures halved), reported
+# beside the measured denominators.
+DATASHEET_TFLOPS = {"bf16": 2250.0, "int8": 4500.0, "fp8": 4500.0}
+
+
 def _bf16_peak(peaks, launch_ms, clocks):
     """(peak TFLOP/s, 'burst'|'sustained') for a fused-kernel launch of this duration."""
     capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
@@ -415,6 +420,7 @@ def _mode_report(w, mode, r, peaks, clocks, gemm):
         out["frac_of_bf16_peak"] = fused / bf16
         out["frac_of_bf16_burst"] = fused / peaks["bf16"]
         out["frac_of_bf16_sustained"] = fused / peaks["bf16_sustained"]
+        out["frac_of_bf16_datasheet"] = fused / DATASHEET_TFLOPS["bf16"]
         return out
     key = "int8" if mode == "int8_qk" else "fp8"
     out["prepass_ms"] = r["kernel_ms"][0]
@@ -423,6 +429,7 @@ def _mode_report(w, mode, r, peaks, clocks, gemm):
     out[f"frac_of_{key}_peak"] = fused / (2.0 * bf16)
     out[f"frac_of_{key}_burst"] = fused / (2.0 * peaks["bf16"])
     out[f"frac_of_{key}_sustained"] = fused / (2.0 * peaks["bf16_sustained"])
+    out[f"frac_of_{key}_datasheet"] = fused / DATASHEET_TFLOPS[key]
     out["frac_of_mixed_peak"] = fused / (bf16 * 4.0 / 3.0)
     alt = gemm.get("int8_tops" if key == "int8" else "fp8_tflops")
     if alt:

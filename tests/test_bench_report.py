@@ -1,0 +1,71 @@
+"""Host logic of bench.py's per-mode report (no GPU): which bf16 peak a fused-kernel launch is
+compared with, and the fractions derived from it."""
+import math
+import os
+import sys
+
+import pytest
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+from attn_workloads import WORKLOADS  # noqa: E402
+
+PEAKS = {"hbm_gbs": 6548.0, "bf16": 1653.3, "bf16_sustained": 1389.5, "source": "measured"}
+CAPPED = {"reasons": ["sw_power_cap"]}
+
+
+def _report(mode, fused_ms, clocks, prepass_ms=0.5, gemm=None):
+    w = WORKLOADS[5]
+    r = {"tflops": 1.0, "ms_per_step": fused_ms + prepass_ms,
+         "kernel_ms": [fused_ms] if mode == "bf16_exact" else [prepass_ms, fused_ms]}
+    return w, bench._mode_report(w, mode, r, PEAKS, clocks, gemm or {})
+
+
+def test_flop_formula_of_the_largest_workload():
+    # 4 * B * Hq * N^2 * d, halved for the causal mask: 140.7 TFLOP for B1 Hq32 N131072 d128
+    w = WORKLOADS[5]
+    assert w.flops() == 4 * 1 * 32 * 131072 ** 2 * 128 // 2
+    assert math.isclose(w.flops() / 1e12, 140.737, rel_tol=1e-4)
+
+
+@pytest.mark.parametrize("fused_ms, clocks, basis", [
+    (115.0, CAPPED, "sustained"),  # a long launch under the power cap: sustained GEMM rate
+    (115.0, {"reasons": []}, "burst"),  # long but never capped
+    (0.5, CAPPED, "burst"),  # a short launch runs at burst clocks whatever the record says
+    (115.0, None, "burst"),  # no clock record
+])
+def test_peak_basis_follows_the_launch(fused_ms, clocks, basis):
+    w, out = _report("int8_qk", fused_ms, clocks)
+    assert out["peak_basis"] == basis
+    bf16 = PEAKS["bf16_sustained"] if basis == "sustained" else PEAKS["bf16"]
+    fused = w.flops() / (fused_ms * 1e-3) / 1e12
+    assert math.isclose(out["fused_tflops"], fused)
+    assert math.isclose(out["frac_of_int8_peak"], fused / (2 * bf16))
+    assert math.isclose(out["frac_of_mixed_peak"], fused / (bf16 * 4 / 3))
+    # both bases are always reported, whichever is the headline one
+    assert math.isclose(out["frac_of_int8_burst"], fused / (2 * PEAKS["bf16"]))
+    assert math.isclose(out["frac_of_int8_sustained"], fused / (2 * PEAKS["bf16_sustained"]))
+
+
+def test_each_mode_against_its_own_datasheet_peak():
+    w, b = _report("bf16_exact", 130.0, CAPPED)
+    assert math.isclose(b["frac_of_bf16_datasheet"], b["fused_tflops"] / 2250.0)
+    assert "prepass_ms" not in b
+    for mode, key in (("int8_qk", "int8"), ("fp8_qk", "fp8")):
+        _, r = _report(mode, 115.0, CAPPED)
+        assert math.isclose(r[f"frac_of_{key}_datasheet"], r["fused_tflops"] / 4500.0)
+
+
+def test_prepass_rate_counts_algorithmic_bytes():
+    w, out = _report("int8_qk", 115.0, CAPPED, prepass_ms=0.5)
+    nq, nk = w.B * w.Hq * w.N * w.d, w.B * w.Hkv * w.N * w.d
+    nbytes = 3 * nq + 3 * nk + 4 * w.B * w.Hq * w.N  # read 16-bit once, write 8-bit codes, lse bias
+    assert math.isclose(out["prepass_gbs"], nbytes / 0.5e-3 / 1e9)
+    assert math.isclose(out["prepass_frac_of_hbm_peak"], out["prepass_gbs"] / PEAKS["hbm_gbs"])
+
+
+def test_measured_library_gemm_is_an_extra_denominator():
+    _, out = _report("int8_qk", 115.0, CAPPED, gemm={"int8_tops": 3051.8})
+    assert math.isclose(out["frac_of_measured_int8_gemm"], out["fused_tflops"] / 3051.8)
+    _, out = _report("fp8_qk", 115.0, CAPPED, gemm={})
+    assert "frac_of_measured_fp8_gemm" not in out
