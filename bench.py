@@ -398,6 +398,17 @@ class _Modes:
 DATASHEET_TFLOPS = {"bf16": 2250.0, "int8": 4500.0, "fp8": 4500.0}
 
 
+# MUFU ex2 results per clock per SM: the softmax's one exponential per score bounds the fused kernel
+# at 4 * d FLOPs (Q K^T and P V for that score) per exponential, whatever N is.
+MUFU_EX2_PER_CLK_SM = 16
+
+
+def _mufu_floor_tflops(d, peaks):
+    if not peaks.get("sms") or not peaks.get("sm_mhz"):
+        return None
+    return 4.0 * d * MUFU_EX2_PER_CLK_SM * peaks["sms"] * peaks["sm_mhz"] * 1e6 / 1e12
+
+
 def _bf16_peak(peaks, launch_ms, clocks):
     """(peak TFLOP/s, 'burst'|'sustained') for a fused-kernel launch of this duration."""
     capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
@@ -416,6 +427,10 @@ def _mode_report(w, mode, r, peaks, clocks, gemm):
     bf16, basis = _bf16_peak(peaks, fused_ms, clocks)
     out = {"tflops": r["tflops"], "ms_per_step": r["ms_per_step"], "fused_ms": fused_ms, "fused_tflops": fused,
            "peak_basis": basis}
+    mufu = _mufu_floor_tflops(w.d, peaks)
+    if mufu:  # the secondary bound: every exponential on MUFU at the sampled SM clock
+        out["mufu_floor_tflops"] = mufu
+        out["frac_of_mufu_floor"] = fused / mufu
     if mode == "bf16_exact":
         out["frac_of_bf16_peak"] = fused / bf16
         out["frac_of_bf16_burst"] = fused / peaks["bf16"]
@@ -457,6 +472,9 @@ def run_native(args, w, world, rank, local):
         results[mode] = mb.time(mode, args.steps, args.warmup, world, sampler if mode == "int8_qk" else None)
     clocks = sampler.stop()
     o, lse = mb.o, mb.lse
+    # the MUFU bound uses the SM count and the median SM clock of the timed region
+    peaks = dict(peaks, sms=torch.cuda.get_device_properties(dev).multi_processor_count,
+                 sm_mhz=(clocks or {}).get("sm_mhz") or (clocks or {}).get("sm_max_mhz"))
 
     # end to end through the public C ABI with host buffers: H2D q,k,v + forward + D2H o, lse
     e2e = None

@@ -69,3 +69,17 @@ def test_measured_library_gemm_is_an_extra_denominator():
     assert math.isclose(out["frac_of_measured_int8_gemm"], out["fused_tflops"] / 3051.8)
     _, out = _report("fp8_qk", 115.0, CAPPED, gemm={})
     assert "frac_of_measured_fp8_gemm" not in out
+
+
+def test_mufu_floor_is_four_d_flops_per_exponential():
+    peaks = dict(PEAKS, sms=148, sm_mhz=1965.0)
+    for cfg in (4, 5):  # d = 64 and d = 128
+        w = WORKLOADS[cfg]
+        r = {"tflops": 1.0, "ms_per_step": 10.0, "kernel_ms": [10.0]}
+        out = bench._mode_report(w, "bf16_exact", r, peaks, None, {})
+        floor = 4 * w.d * 16 * 148 * 1965e6 / 1e12  # 1.19 PFLOP/s at d = 64, 2.38 at d = 128
+        assert math.isclose(out["mufu_floor_tflops"], floor)
+        assert math.isclose(out["frac_of_mufu_floor"], out["fused_tflops"] / floor)
+    # without an SM count or clock the bound is left out rather than guessed
+    _, out = _report("int8_qk", 115.0, CAPPED)
+    assert "mufu_floor_tflops" not in out
