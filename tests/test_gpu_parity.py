@@ -92,6 +92,9 @@ SMALL = [
     (1, 2, 2, 640, 128, True, "bf16", "k_offset"),   # several 256-row blocks, no tail
     (1, 8, 2, 383, 128, False, "fp16", "k_offset"),
     (1, 2, 1, 1000, 64, False, "bf16", "normal"),
+    # many work items over several SMs with a ragged tail: 8 per head, 16 heads, 4:1 GQA
+    (2, 8, 2, 1999, 128, True, "bf16", "k_offset"),
+    (1, 6, 3, 1537, 64, True, "fp16", "outlier_channels"),
 ]
 
 
@@ -203,6 +206,25 @@ def test_full_size_sampled_rows(ta, cfg, mode):
         c_emu = cosine(np.concatenate(Oe_all), np.concatenate(O_all))
         assert c_gpu >= min(INT8_COS, c_emu - 1e-3), (c_gpu, c_emu)
     assert torch.isfinite(o).all()
+
+
+@pytest.mark.parametrize("scale", [0.02, 0.35])
+@pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk"])
+def test_explicit_softmax_scale(ta, mode, scale):
+    """A scale other than 1/sqrt(d): 0.35 makes the scores four times larger (more running-max
+    moves), 0.02 flattens them; the oracle gets the same scale."""
+    w = Workload("t", 1, 4, 2, 700, 128, True, "bf16", "k_offset", 99800)
+    q, k, v = make_inputs(w)
+    o, l = ta.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, scale=scale, mode=mode)
+    torch.cuda.synchronize()
+    assert ta.attn_check_status() == 0
+    o, l = _np(o), l.cpu().numpy().astype(np.float64)
+    O, L = oracle.attention(q, k, v, scale, True)
+    if mode == "bf16_exact":
+        assert_bf16(o, l, O, L, f"scale {scale}")
+    else:
+        Oe, Le = emulated(q, k, v, True, scale)
+        assert_int8(o, l, O, L, Oe, Le, f"scale {scale}")
 
 
 @pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk"])
