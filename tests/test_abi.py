@@ -173,3 +173,23 @@ def test_binding_refuses_tensors_on_two_devices():
         binding._device_of(a0, _FakeTensor("cpu"))
     with pytest.raises(ValueError, match="no CUDA tensor"):
         binding._device_of(None, None)
+
+
+def test_plain_c_consumer_builds_and_runs(lib, tmp_path):
+    """The header is usable from C99 on its own: tests/c_consumer.c includes only it, links the
+    shared library, and checks the host-side calls (no device work)."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    from tiled_attention_22_b200 import binding
+
+    libdir = os.path.dirname(binding.LIB_PATH)
+    exe = str(tmp_path / "c_consumer")
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_consumer.c"), "-L", libdir, "-ltiled_attention",
+                    "-Wl,-rpath," + libdir, "-lm", "-o", exe], check=True, capture_output=True, text=True)
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip().endswith("OK"), run.stdout + run.stderr
