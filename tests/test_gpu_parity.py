@@ -227,6 +227,21 @@ def test_explicit_softmax_scale(ta, mode, scale):
         assert_int8(o, l, O, L, Oe, Le, f"scale {scale}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk", "fp8_qk"])
+def test_output_without_lse_equals_output_with_lse(ta, mode, d):
+    """lse = NULL skips the lse write (and, in the 8-bit modes, the lse-bias load); O must be the
+    same bytes as with lse requested (bf16 at d = 128 takes the persistent kernel)."""
+    w = Workload("t", 2, 4, 2, 777, d, True, "bf16", "k_offset", 99900 + d)
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    o1, l1 = ta.attn_fwd(q, k, v, causal=True, mode=mode)
+    o2, l2 = ta.attn_fwd(q, k, v, causal=True, mode=mode, lse=False)
+    torch.cuda.synchronize()
+    assert ta.attn_check_status() == 0
+    assert l2 is None and l1 is not None and torch.isfinite(l1).all()
+    assert torch.equal(o1, o2)
+
+
 @pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk"])
 def test_zero_inputs(ta, mode):
     z = torch.zeros((1, 2, 300, 128), dtype=torch.bfloat16)
