@@ -202,3 +202,17 @@ def test_workspace_reuse_across_calls(ta):
         check(_np(o), l.cpu().numpy().astype(np.float64), O, L, seen, f"lens {lens} ctas {ctas}")
     # the per-unit arrival counters (the first U int32 of the workspace) are back at zero
     assert not ws[:3 * 4 * 4].cpu().numpy().any()
+
+
+def test_output_without_lse_equals_output_with_lse(ta):
+    """lse = NULL only skips the lse write: the split-KV pieces are still merged by their own
+    log-sum-exp in the workspace, so O is the same bytes (pieces over several CTAs, causal drafts,
+    one sequence with an empty cache)."""
+    q, k, v, lt = _inputs(3, 16, 4, 4, 3000, "bf16", "k_offset", 93000, [3000, 1777, 0])
+    qc, kc, vc, lc = q.cuda(), k.cuda(), v.cuda(), lt.cuda()
+    o1, l1 = ta.attn_decode(qc, kc, vc, lc, causal=True, num_ctas=9)
+    o2, l2 = ta.attn_decode(qc, kc, vc, lc, causal=True, num_ctas=9, lse=False)
+    torch.cuda.synchronize()
+    assert ta.attn_check_status() == 0
+    assert l2 is None and l1 is not None
+    assert torch.equal(o1, o2)

@@ -139,3 +139,17 @@ def test_apb_workload_full_size(ta, cfg):
         O, Lr = oracle.attention_prefix(q[:, h:h + 1], k[:, h // (w.Hq // w.Hkv):h // (w.Hq // w.Hkv) + 1],
                                         v[:, h // (w.Hq // w.Hkv):h // (w.Hq // w.Hkv) + 1], w.scale, lim, rows=rows)
         check(o[:, h:h + 1, rows], l[:, h:h + 1, rows], O, Lr, f"{w.name} head {h}")
+
+
+def test_output_without_lse_equals_output_with_lse(ta):
+    """lse = NULL only skips the lse write (rows with limit 0 still get O = 0)."""
+    q, k, v = _qkv(1, 4, 2, 600, 900, 128, "bf16", 62500)
+    lim = torch.as_tensor(np.concatenate([np.zeros(40), np.arange(1, 561) + 300]).astype(np.int32)).cuda()
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o1, l1 = ta.attn_fwd_prefix_masked(qc, kc, vc, lim)
+    o2, l2 = ta.attn_fwd_prefix_masked(qc, kc, vc, lim, lse=False)
+    torch.cuda.synchronize()
+    assert ta.attn_check_status() == 0
+    assert l2 is None and l1 is not None
+    assert torch.equal(o1, o2)
+    assert (o2[:, :, :40] == 0).all()
