@@ -208,6 +208,39 @@ def test_full_size_sampled_rows(ta, cfg, mode):
     assert torch.isfinite(o).all()
 
 
+def test_tensors_beyond_2_31_elements(ta):
+    """Q and O hold more than 2^31 elements: 136 query heads (8 kv heads) of 131072 tokens at
+    d = 128, 2.28 G elements each (about 12 GB on the device with K, V, lse and the INT8
+    workspace).  Head 128 starts at element 2^31, so an element offset computed in 32 bits would
+    wrap there.  Sampled rows of heads on both sides of that boundary, and of the last head,
+    against the oracle in both modes."""
+    w = Workload("t", 1, 136, 8, 131072, 128, True, "bf16", "k_offset", 99950)
+    q, k, v = make_inputs(w)
+    assert q.numel() > 2 ** 31
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    rng = np.random.default_rng(31)
+    rows = sorted(set([0, 1, 127, 128, 255, 256, w.N // 2, w.N - 257, w.N - 129, w.N - 128, w.N - 1]
+                      + [int(x) for x in rng.integers(0, w.N, 5)]))
+    G = w.Hq // w.Hkv
+    for mode in ("bf16_exact", "int8_qk"):
+        o, l = ta.attn_fwd(qd, kd, vd, causal=True, mode=mode)
+        torch.cuda.synchronize()
+        assert ta.attn_check_status() == 0
+        for h in (0, 127, 128, 135):
+            g = h // G
+            qs, ks, vs = q[:, h:h + 1], k[:, g:g + 1], v[:, g:g + 1]
+            og = _np(o[0, h, rows])[None, None]
+            lg = l[0, h, rows].cpu().numpy().astype(np.float64)[None, None]
+            O, L = oracle.attention(qs, ks, vs, w.scale, True, rows=rows)
+            if mode == "bf16_exact":
+                assert_bf16(og, lg, O, L, f"head {h}")
+            else:
+                Oe, Le = emulated(qs, ks, vs, True, w.scale, rows=rows)
+                assert_int8(og, lg, O, L, Oe, Le, f"head {h}")
+        del o, l
+        torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("scale", [0.02, 0.35])
 @pytest.mark.parametrize("mode", ["bf16_exact", "int8_qk"])
 def test_explicit_softmax_scale(ta, mode, scale):
