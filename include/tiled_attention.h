@@ -316,6 +316,14 @@ int attn_merge_lse(float* o_acc, float* lse_acc, const void* o_part, const float
                    void* o_out, long long rows, int d, int dtype, int first, void* stream);
 
 /*
+ * attn_test_host_pieces - test hook: the pieces attn_fwd_host cuts the B*Hq query heads into, as
+ * cut points cuts[0] = 0 < cuts[1] < ... < cuts[n] = B*Hq; returns n (at most 16) or a negative
+ * ATTN_ERR_* code (the shape checks of attn_fwd; cuts NULL or max_cuts < 17 is ATTN_ERR_ARG).
+ * Host only: nothing is launched.
+ */
+int attn_test_host_pieces(int B, int Hq, int Hkv, int N, int d, int* cuts, int max_cuts);
+
+/*
  * attn_test_wait_timeout - test hook for failure detection.  Launches one tiny kernel whose single
  * thread waits on an mbarrier that nothing ever completes, with a limit of `limit_us`
  * microseconds (1..1000000).  The wait gives up, sets the device status word and the kernel

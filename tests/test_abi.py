@@ -193,3 +193,40 @@ def test_plain_c_consumer_builds_and_runs(lib, tmp_path):
                     "-Wl,-rpath," + libdir, "-lm", "-o", exe], check=True, capture_output=True, text=True)
     run = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0 and run.stdout.strip().endswith("OK"), run.stdout + run.stderr
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 32, 8, 131072), (2, 32, 8, 8192), (4, 32, 32, 4096), (2, 24, 24, 16384),  # the named workloads
+    (1, 4, 2, 500), (3, 6, 3, 333), (2, 8, 8, 1024), (1, 4, 1, 256), (2, 8, 2, 2048),  # the GPU test shapes
+    (1, 1, 1, 1), (1, 2, 1, 4), (1, 3, 3, 334), (5, 8, 1, 12), (64, 16, 4, 100), (1, 128, 2, 96),
+])
+def test_host_buffer_pieces(lib, shape):
+    """The query-head pieces of attn_fwd_host: contiguous cover of all B*Hq heads; each piece
+    whole (batch, kv head) units or heads inside one unit (so one kernel call can do it); every
+    piece's lse slice 16-byte aligned; at most 10 pieces; single heads (or single units when
+    Hq == Hkv) at both ends whenever N % 4 == 0."""
+    from tiled_attention_22_b200 import binding
+
+    B, Hq, Hkv, N = shape
+    cuts = binding.attn_test_host_pieces(B, Hq, Hkv, N, 128)
+    heads, G = B * Hq, Hq // Hkv
+    assert cuts[0] == 0 and cuts[-1] == heads
+    assert all(a < b for a, b in zip(cuts, cuts[1:]))
+    assert len(cuts) - 1 <= 10
+    for a, b in zip(cuts, cuts[1:]):
+        whole = a % G == 0 and (b - a) % G == 0
+        assert whole or a // G == (b - 1) // G, (a, b)
+        assert (a * N * 4) % 16 == 0, (a, "lse slice not 16-byte aligned")
+    if N % 4 == 0 and heads > 1:
+        first, last = cuts[1] - cuts[0], cuts[-1] - cuts[-2]
+        assert first == (1 if G > 1 else G) and last == (1 if G > 1 else G)
+
+
+def test_host_buffer_pieces_reject_bad_shapes(lib):
+    from tiled_attention_22_b200 import binding
+
+    for args, code in (((1, 3, 2, 128, 128), -1), ((1, 2, 2, 128, 96), -2), ((0, 2, 2, 128, 64), -1)):
+        with pytest.raises(binding.AttnError) as e:
+            binding.attn_test_host_pieces(*args)
+        assert e.value.code == code
+    assert lib.attn_test_host_pieces(1, 2, 2, 128, 64, None, 17) == -1

@@ -32,6 +32,7 @@ from .binding import (  # noqa: F401
     attn_quant_smooth_k_fp8,
     attn_quant_smooth_k_noalloc,
     attn_test_exp2,
+    attn_test_host_pieces,
     attn_test_wait_timeout,
     attn_workspace_bytes,
     exported_symbols,

@@ -48,6 +48,7 @@ _SIGNATURES = {
     "attn_check_status": (_i, []),
     "attn_error_string": (ctypes.c_char_p, [_i]),
     "attn_last_cuda_error": (ctypes.c_char_p, []),
+    "attn_test_host_pieces": (_i, [_i, _i, _i, _i, _i, _vp, _i]),
     "attn_test_wait_timeout": (_i, [_i, _vp]),
     "attn_test_exp2": (_i, [_vp, _vp, _i, _i, _vp]),
 }
@@ -442,6 +443,15 @@ def attn_check_status() -> int:
 
 def attn_error_string(code: int) -> str:
     return load_library().attn_error_string(code).decode()
+
+
+def attn_test_host_pieces(B, Hq, Hkv, N, d):
+    """The query-head cut points attn_fwd_host uses for this shape (a list of ints)."""
+    buf = (ctypes.c_int * 17)()
+    n = load_library().attn_test_host_pieces(B, Hq, Hkv, N, d, ctypes.cast(buf, ctypes.c_void_p), 17)
+    if n < 0:
+        raise AttnError(n, "attn_test_host_pieces")
+    return list(buf[:n + 1])
 
 
 def attn_test_wait_timeout(limit_us: int, stream=None) -> None:

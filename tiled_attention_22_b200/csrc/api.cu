@@ -380,6 +380,43 @@ int attn_probe_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int H
   return ATTN_OK;
 }
 
+// The pieces attn_fwd_host cuts B*Hq query heads into, as cut points cut[0] = 0 < cut[1] < ... <
+// cut[n] = B*Hq (n <= kMaxPieces, returned).  A piece is either whole (batch, kv head) units
+// (G = Hq/Hkv heads each) or a run of query heads inside one unit.  When N % 4 == 0 (every
+// head's lse slice 16-byte aligned) the first and last pieces are one query head each (one unit
+// when G = 1) and the units between form up to six pieces; otherwise up to 8 runs of whole
+// units, 4-unit aligned when a unit's lse slice is not 16-byte aligned.
+constexpr int kMaxPieces = 16;
+static int host_pieces(int B, int Hq, int Hkv, int N, int* cut) {
+  const int G = Hq / Hkv;
+  const int units = B * Hkv, heads = B * Hq;
+  int c[kMaxPieces + 8];
+  int nc = 0;
+  if (N % 4 == 0) {
+    c[nc++] = 0;
+    c[nc++] = 1;
+    c[nc++] = G;
+    const int mid = units - 2 > 0 ? units - 2 : 0;  // units strictly between the first and last
+    const int nm = mid < 6 ? mid : 6;
+    for (int i = 1; i < nm; ++i) c[nc++] = (1 + (int)((long long)mid * i / nm)) * G;
+    c[nc++] = heads - G;
+    c[nc++] = heads - 1;
+    c[nc++] = heads;
+  } else {
+    const int align_units = ((size_t)G * N * 4 % 16 == 0) ? 1 : 4;
+    const int n8 = units < 8 ? units : 8;
+    for (int i = 0; i <= n8; ++i) c[nc++] = (int)((long long)units * i / n8) / align_units * align_units * G;
+    c[nc++] = heads;
+  }
+  std::sort(c, c + nc);
+  int n = 0;
+  for (int i = 0; i < nc; ++i) {
+    if (i > 0 && c[i] == c[i - 1]) continue;
+    cut[n++] = c[i];
+  }
+  return n - 1;
+}
+
 int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, void* dq, void* dk, void* dv,
                   void* do_, float* dlse, int B, int Hq, int Hkv, int N, int d, int causal, float scale, int mode,
                   int dtype, void* workspace, size_t ws_bytes, void* stream) {
@@ -395,45 +432,15 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
   // O and lse slices are contiguous, in unit order, in every [B, H, N, d] tensor.  A run of whole
   // units is one problem with B' = 1, Hq' = n*G, Hkv' = n, and a run of query heads inside one
   // unit is one with B' = 1, Hq' = n, Hkv' = 1 (the unit's K and V); either gives every output row
-  // the same arithmetic as the whole call.  The work is cut into pieces of query heads; piece c's
-  // inputs are copied in on a helper stream while piece c-1 computes on the caller's stream, and
-  // its outputs are copied out on a second helper stream.  Only the first piece's input copy and
-  // the last piece's output copy are not hidden behind compute, so when every head's lse slice is
-  // 16-byte aligned (N % 4 == 0) the first and last pieces are a single query head (a single unit
-  // when G = 1) and the units between them form up to six pieces.  Otherwise pieces are up to 8
-  // runs of whole units, 4-unit aligned when a unit's lse slice is not 16-byte aligned.
+  // the same arithmetic as the whole call.  The work is cut into pieces of query heads
+  // (host_pieces); piece c's inputs are copied in on a helper stream while piece c-1 computes on
+  // the caller's stream, and its outputs are copied out on a second helper stream.  Only the first
+  // piece's input copy and the last piece's output copy are not hidden behind compute, which is
+  // why those two pieces are kept small.
   const int G = Hq / Hkv;
-  const int units = B * Hkv, heads = B * Hq;
   const size_t q_head = (size_t)N * d * 2, kv_unit = (size_t)N * d * 2, l_head = (size_t)N * 4;
-  constexpr int kMaxPieces = 16;
   int cut[kMaxPieces + 1];
-  int npiece = 0;
-  {
-    int c[kMaxPieces + 8];
-    int nc = 0;
-    if (N % 4 == 0) {
-      c[nc++] = 0;
-      c[nc++] = 1;
-      c[nc++] = G;
-      const int mid = units - 2 > 0 ? units - 2 : 0;  // units strictly between the first and last
-      const int nm = mid < 6 ? mid : 6;
-      for (int i = 1; i < nm; ++i) c[nc++] = (1 + (int)((long long)mid * i / nm)) * G;
-      c[nc++] = heads - G;
-      c[nc++] = heads - 1;
-      c[nc++] = heads;
-    } else {
-      const int align_units = ((size_t)G * l_head % 16 == 0) ? 1 : 4;
-      const int n8 = units < 8 ? units : 8;
-      for (int i = 0; i <= n8; ++i) c[nc++] = (int)((long long)units * i / n8) / align_units * align_units * G;
-      c[nc++] = heads;
-    }
-    std::sort(c, c + nc);
-    for (int i = 0; i < nc; ++i) {
-      if (i > 0 && c[i] == c[i - 1]) continue;
-      cut[npiece++] = c[i];
-    }
-    npiece -= 1;  // cut[0..npiece] bound npiece pieces
-  }
+  const int npiece = host_pieces(B, Hq, Hkv, N, cut);
   cudaStream_t s_in = nullptr, s_out = nullptr;
   cudaEvent_t ev_in[kMaxPieces] = {}, ev_done[kMaxPieces] = {};
   auto cleanup = [&]() {
@@ -599,6 +606,13 @@ int attn_check_status(void) {
 
 // Test hook for failure detection: one thread waits on an mbarrier that nothing ever completes,
 // with a limit of `limit_us` microseconds, so the bounded-wait path runs without faulting the GPU.
+int attn_test_host_pieces(int B, int Hq, int Hkv, int N, int d, int* cuts, int max_cuts) {
+  if (!cuts || max_cuts < kMaxPieces + 1) return ATTN_ERR_ARG;
+  int rc = check_shape(B, Hq, Hkv, N, d);
+  if (rc) return rc;
+  return host_pieces(B, Hq, Hkv, N, cuts);
+}
+
 int attn_test_wait_timeout(int limit_us, void* stream) {
   if (limit_us < 1 || limit_us > 1000000) return ATTN_ERR_ARG;
   wait_forever_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((unsigned long long)limit_us * 1000ull);
